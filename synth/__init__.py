@@ -1,0 +1,163 @@
+"""Seeded synthetic inputs shared by the oracle side and the CUDA side.
+
+Holds none of the attention method's arithmetic: only the workload shapes and
+the recipes that draw BF16 Q/K/V (``gen.c``).  The five workloads mirror the
+shapes of the H3 video-diffusion attention described on the pages:
+
+* ``fixed_q128_kv192``: the fixed single-tile shape of the aligned numerical
+  prototype ("Phase 2B Aligned Numerical Prototype", Decision): B=1, H=1,
+  Tq=128, Tkv=192, D=128, N(0,1) values.
+* ``selfattn_h8_t4096``: B=1, H=8, T=4096; K has a per-channel offset drawn
+  from N(0, 4) (std 2) to exercise K mean-smoothing.
+* ``ragged_h16_t9453``: B=1, H=16, T=9453 (not a multiple of 64 or 128); Q/K
+  RMS-normalised per (token, head) and scaled by gamma ~ N(1, 0.1).
+* ``h3_t37810_h32``: the H3 packed video+text sequence of the representative
+  workload ("H3 Performance Roadmap", Measured GB10 Baseline: 37,810 packed
+  tokens), H=32, D=128, Q/K RMS-normed with gamma.
+* ``h3_packed_b2_t37810``: the same shape with batch 2 read from one packed
+  [2, T, 3, H, D] QKV buffer, output into [2, T, H*D].
+
+N(mu, v) names a normal with variance v.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libsynth.so")
+_SRC = os.path.join(_HERE, "gen.c")
+
+NORMAL, OFFSET, RMSNORM = 0, 1, 2
+STREAM_Q, STREAM_K, STREAM_V, STREAM_GAMMA_Q, STREAM_GAMMA_K, STREAM_OFFSET_K = range(6)
+
+
+def build(force: bool = False) -> str:
+    """Compile gen.c into libsynth.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + ".tmp"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.synth_normal_f32.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64,
+                                         ctypes.c_uint32, ctypes.c_double, ctypes.c_double]
+        lib.synth_fill_bf16.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_int64] * 3 + [
+            ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_void_p]
+        _lib = lib
+    return _lib
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Tq: int
+    Tkv: int
+    H: int
+    D: int
+    recipe: str          # "normal", "k_offset" or "rmsnorm"
+    seed: int
+    packed: bool = False  # Q/K/V read from one [B,T,3,H,D] buffer, out [B,T,H*D]
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.D))
+
+    @property
+    def ops(self) -> float:
+        """Algorithmic tensor operations of one call: 2*D per score for QK and 2*D for PV."""
+        return 4.0 * self.B * self.Tq * self.Tkv * self.H * self.D
+
+
+WORKLOADS = {
+    "fixed_q128_kv192": Workload("fixed_q128_kv192", 1, 128, 192, 1, 128, "normal", 73021),
+    "selfattn_h8_t4096": Workload("selfattn_h8_t4096", 1, 4096, 4096, 8, 128, "k_offset", 4096),
+    "ragged_h16_t9453": Workload("ragged_h16_t9453", 1, 9453, 9453, 16, 128, "rmsnorm", 9453),
+    "h3_t37810_h32": Workload("h3_t37810_h32", 1, 37810, 37810, 32, 128, "rmsnorm", 37810),
+    "h3_packed_b2_t37810": Workload("h3_packed_b2_t37810", 2, 37810, 37810, 32, 128, "rmsnorm", 37811,
+                                    packed=True),
+}
+
+
+def normal_f32(n: int, seed: int, stream: int, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
+    out = np.empty(n, dtype=np.float32)
+    _load().synth_normal_f32(out.ctypes.data, n, seed, stream, mean, std)
+    return out
+
+
+def fill_bf16(out: np.ndarray, B: int, T: int, H: int, D: int, strides, seed: int, stream: int,
+              kind: int = NORMAL, mean: float = 0.0, std: float = 1.0, vec: np.ndarray | None = None,
+              offset_elems: int = 0):
+    """Fill the logical [B,T,H,D] view at ``out.flat[offset_elems:]`` with element strides (sb, st, sh).
+
+    ``out`` is a C-contiguous uint16 array (BF16 bit patterns) that must span the whole view.
+    """
+    assert out.dtype == np.uint16 and out.flags.c_contiguous
+    assert D <= 1024
+    sb, st, sh = strides
+    last = offset_elems + (B - 1) * sb + (T - 1) * st + (H - 1) * sh + D
+    assert 0 <= offset_elems and last <= out.size
+    if kind != NORMAL:
+        assert vec is not None and vec.dtype == np.float32 and vec.size == H * D
+        vec = np.ascontiguousarray(vec)
+    _load().synth_fill_bf16(out.ctypes.data + 2 * offset_elems, B, T, H, D, sb, st, sh, seed, stream,
+                            kind, mean, std, None if vec is None else vec.ctypes.data)
+
+
+def _fill_tensor(out, w: Workload, T: int, strides, which: str, offset_elems: int = 0):
+    stream = {"q": STREAM_Q, "k": STREAM_K, "v": STREAM_V}[which]
+    H, D = w.H, w.D
+    kw = dict(offset_elems=offset_elems)
+    if which == "v" or w.recipe == "normal" or (w.recipe == "k_offset" and which == "q"):
+        fill_bf16(out, w.B, T, H, D, strides, w.seed, stream, **kw)
+    elif w.recipe == "k_offset":
+        off = normal_f32(H * D, w.seed, STREAM_OFFSET_K, 0.0, 2.0)
+        fill_bf16(out, w.B, T, H, D, strides, w.seed, stream, OFFSET, vec=off, **kw)
+    elif w.recipe == "rmsnorm":
+        gstream = STREAM_GAMMA_Q if which == "q" else STREAM_GAMMA_K
+        gamma = normal_f32(H * D, w.seed, gstream, 1.0, float(np.sqrt(0.1)))
+        fill_bf16(out, w.B, T, H, D, strides, w.seed, stream, RMSNORM, vec=gamma, **kw)
+    else:
+        raise ValueError(w.recipe)
+
+
+def make_separate(w: Workload):
+    """Q [B,Tq,H,D], K and V [B,Tkv,H,D], contiguous uint16 BF16 bit patterns."""
+    out = {}
+    for which, T in (("q", w.Tq), ("k", w.Tkv), ("v", w.Tkv)):
+        a = np.empty((w.B, T, w.H, w.D), dtype=np.uint16)
+        _fill_tensor(a, w, T, (T * w.H * w.D, w.H * w.D, w.D), which)
+        out[which] = a
+    return out
+
+
+def make_packed(w: Workload):
+    """One packed [B,T,3,H,D] uint16 buffer (Tq == Tkv); slot 0 = Q, 1 = K, 2 = V."""
+    assert w.Tq == w.Tkv
+    T, H, D = w.Tq, w.H, w.D
+    buf = np.empty((w.B, T, 3, H, D), dtype=np.uint16)
+    strides = (T * 3 * H * D, 3 * H * D, D)
+    for slot, which in enumerate(("q", "k", "v")):
+        _fill_tensor(buf, w, T, strides, which, offset_elems=slot * H * D)
+    return buf
+
+
+def make_inputs(w: Workload):
+    """Inputs for a workload: dict with 'q','k','v' logical [B,T,H,D] views (and 'packed' if packed)."""
+    if w.packed:
+        buf = make_packed(w)
+        return {"packed": buf, "q": buf[:, :, 0], "k": buf[:, :, 1], "v": buf[:, :, 2]}
+    return make_separate(w)
