@@ -1,0 +1,350 @@
+"""Benchmark: quantized attention effective TOPS and ms per call on B200.
+
+One step = one ``h3attn_forward`` call (K smoothing + Q/K/V quantization +
+the fused attention mainloop) over the H3-shaped packed video+text sequence
+(B=1, T=37,810, H=32, D=128).  Effective TOPS = 4*B*Tq*Tkv*H*D / time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own copy of the workload on its own
+GPU (independent problems, weak scaling, no data-path collective); timing is
+the max over ranks.  ``--impl reference`` times the CPU oracle on the host
+cores on a bounded sample of the same workload (rank 0 only).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "quantized attention effective TOPS and ms/call at T=37,810, H=32, D=128 (1xB200)"
+UNIT = "TOPS"
+DEFAULT_WORKLOAD = "h3_t37810_h32"
+KERNEL_SOURCES = ["quantized_attention_video_b200/csrc/attention.cu", "quantized_attention_video_b200/csrc/sm100_ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-rows", type=int, default=48)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H (a smaller case of the same kernel for profiler captures)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def config_of(w: synth.Workload, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "Tq": w.Tq, "Tkv": w.Tkv, "H": w.H, "D": w.D,
+            "layout": "packed [B,T,3,H,D] in, [B,T,H*D] out" if w.packed else "separate [B,T,H,D] in and out",
+            "inputs": f"seeded synthetic ({w.recipe}), seed {w.seed}",
+            "l2": "inputs + workspace > 126 MB L2; no flush between steps",
+            "parallelism": f"independent replica per GPU x{world}" if world > 1 else "single GPU"}
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def cpu_oracle_sample(w: synth.Workload, rows_per_head: int, x=None):
+    """Time the oracle on a bounded sample: quantize of one head plus attention of
+    `rows_per_head` query rows of that head.  Returns (TOPS, seconds, threads, text)."""
+    import oracle
+    oracle.build()
+    if x is None:
+        x = synth.make_inputs(w)
+    q, k, v = (x[n][:, :, :1] for n in ("q", "k", "v"))
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    z = oracle.quantize(q, k, v)
+    t_quant = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rows = np.stack([np.zeros(rows_per_head, int), np.zeros(rows_per_head, int),
+                     np.sort(rng.choice(w.Tq, rows_per_head, replace=False))], axis=1)
+    t0 = time.perf_counter()
+    oracle.attend_rows(z, w.scale, 128, rows)
+    t_rows = time.perf_counter() - t0
+    # the quantize pass is shared by all Tq rows of the head; charge its share
+    secs = t_rows + t_quant * rows_per_head / w.Tq
+    ops = 4.0 * rows_per_head * w.Tkv * w.D
+    text = (f"{w.name}: quantize of 1 of {w.B * w.H} heads ({t_quant:.2f} s, charged pro rata) + attention "
+            f"of {rows_per_head} random query rows of it ({t_rows:.2f} s) on {threads} threads")
+    return ops / secs / 1e12, secs, threads, text
+
+
+def run_reference(args, w):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    K = max(1, args.steps)
+    vals = []
+    x = synth.make_inputs(w)
+    info = None
+    if args.warmup > 0:
+        cpu_oracle_sample(w, max(2, args.cpu_sample_rows // 8), x)
+    for _ in range(K):
+        tops, secs, threads, text = cpu_oracle_sample(w, max(2, args.cpu_sample_rows // 4), x)
+        vals.append(tops)
+        info = (threads, text)
+    value = statistics.median(vals)
+    ms = 4.0 * w.B * w.Tq * w.Tkv * w.H * w.D / (value * 1e12) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic",
+            "config": config_of(w, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": info[0], "kind": "oracle", "sample": info[1]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "note": "CPU oracle on host cores; ms_per_step extrapolates the sampled rate to the whole call"}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ clocks ----
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else f"/tmp/h3attn_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [s.strip() for s in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax = float(p[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, p[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def traffic_record():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256()
+    for src in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, src), "rb").read())
+    if rec.get("kernel_sha256") != h.hexdigest():
+        return None
+    return rec
+
+
+# --------------------------------------------------------------- GPU arm ----
+def run_ours(args, w):
+    import torch
+    import quantized_attention_video_b200 as h3
+    from quantized_attention_video_b200 import build as h3build
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if rank == 0 or not os.path.exists(h3build.SO):
+        h3build.build()
+    if dist is not None:
+        dist.barrier()
+    h3.lib()
+
+    x = synth.make_inputs(w)
+    ops = w.ops
+    dev = torch.device("cuda", local)
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    if w.packed:
+        buf = to_dev(x["packed"])
+        q, k, v = buf[:, :, 0], buf[:, :, 1], buf[:, :, 2]
+        out_flat = torch.empty(w.B, w.Tq, w.H * w.D, dtype=torch.bfloat16, device=dev)
+        out = out_flat.view(w.B, w.Tq, w.H, w.D)
+    else:
+        q, k, v = (to_dev(x[n]) for n in ("q", "k", "v"))
+        out = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device=dev)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        h3.h3attn_quantize_qkv(q, k, v, ws, stream)
+        h3.h3attn_attend(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if h3.h3attn_check_status(ws, stream) != h3.OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        ev[i][0].record(stream)
+        h3.h3attn_quantize_qkv(q, k, v, ws, stream)
+        ev[i][1].record(stream)
+        h3.h3attn_attend(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    if h3.h3attn_check_status(ws, stream) != h3.OK:
+        raise RuntimeError("device status not OK after the timed steps")
+
+    def max_over_ranks(val):
+        if dist is None:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    total_ms = max_over_ranks(total_ms)
+    ms_step = total_ms / K
+    value = world * ops / (ms_step * 1e-3) / 1e12
+    attn_avg = max_over_ranks(statistics.mean(attn_ms))
+    quant_avg = max_over_ranks(statistics.mean(quant_ms))
+
+    # ------------------------------------------------ end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        if w.packed:
+            h_in = [torch.from_numpy(x["packed"].view(np.int16)).pin_memory()]
+            d_in = [buf]
+        else:
+            h_in = [torch.from_numpy(np.ascontiguousarray(x[n]).view(np.int16)).pin_memory() for n in ("q", "k", "v")]
+            d_in = [q, k, v]
+        h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            for hsrc, ddst in zip(h_in, d_in):
+                ddst.view(torch.int16).copy_(hsrc, non_blocking=True)
+            h3.h3attn_forward(q, k, v, w.scale, out, ws, stream) if w.Tq == w.Tkv else \
+                h3.h3attn_forward_ex(q, k, v, w.scale, out, ws, stream)
+            h_out.copy_(out, non_blocking=True)
+
+        Ke = max(3, K // 4)
+        for _ in range(2):
+            e2e_step()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke)
+        e2e = {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms, "steps": Ke,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "pinned host Q/K/V -> device, h3attn_forward, device out -> pinned host"}
+
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    if "bf16_tflops_sustained" in peaks:
+        peak = 2.0 * peaks["bf16_tflops_sustained"]
+        peak_note = "of measured: 2 x bf16_tflops_sustained (nominal 8-bit/bf16 ratio 2), kernel timed inside a long loop"
+    else:
+        peak = 2.0 * 1400.0
+        peak_note = "of fallback: 2 x 1.4 PFLOP/s sustained bf16"
+    achieved = ops / (attn_avg * 1e-3) / 1e12
+    tr = traffic_record()
+    roofline = {"bound": "tensor", "kernel": "attn_sm100_kernel", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_note,
+                "algorithmic_ops_per_launch": ops,
+                "traffic": None if tr is None else tr["dram_bytes_per_launch_full"],
+                "quantize_ms": quant_avg, "attention_ms": attn_avg,
+                "quantize_gbs": (10 * w.B * w.Tkv * w.H * w.D + 2 * w.B * w.Tq * w.H * w.D
+                                 + 3 * w.B * w.Tkv * w.H * w.D) / (quant_avg * 1e-3) / 1e9}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tops, secs, threads, text = cpu_oracle_sample(w, args.cpu_sample_rows, x)
+        cpu = {"value": tops, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": text}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic", "config": config_of(w, world),
+            "clocks": clk, "gpu_launches": 4 * K, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_h{args.heads}", H=args.heads)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * h3attn — quantized dense self-attention for the H3 video-diffusion block,
+ * native to NVIDIA B200 (sm_100a).  C ABI of libh3attn.so.
+ *
+ * The operation is the dense Sage-compatible attention of "H3 Performance
+ * Roadmap", Phase 4: Dense Sage-Compatible Attention: it consumes strided BSHD
+ * Q/K/V views directly, keeps the SageAttention 2.2.0 numerical policy
+ * (per-warp INT8 Q/K with K smoothing, FP8 V, FP32 accumulation) and writes
+ * token-major output that the out-projection reads without a copy.  Its
+ * numerical checkpoints are those of "Phase 2B Aligned Numerical Prototype",
+ * Exactness (INT32-to-FP32 QK scores, per-epoch online-softmax m and d, FP8
+ * E4M3 probability words, FP32 RO, final reciprocal, BF16 output).
+ *
+ * Policy implemented (D = 128; all divisions and products correctly rounded):
+ *   km[b,h,c]   = mean over the Tkv keys of K[b,:,h,c]  (FP64 sums, FP32 result)
+ *   Q groups    : 32 tokens per (b,h); sq = amax/127; q8 = clamp(rne(x*(127/amax)), +-127)
+ *   K groups    : 64 tokens per (b,h), on K - km, same rule -> k8, sk
+ *   V channels  : sv = amax_c/448;  v8 = e4m3_rne_satfinite(v * (448/amax_c))
+ *   scores      : acc = sum_c q8*k8 (exact INT32);  t = float(acc) * ((sq*sk) * c),
+ *                 c = float(softmax_scale * log2(e));  keys >= Tkv masked
+ *   per 128-key tile: m' = max(m, max t); alpha = 2^(m - m'); p = 2^(t - m');
+ *                 d = d*alpha + sum p;  p8 = e4m3(448*p);  RO = RO*alpha + p8 x v8
+ *   out         = bf16((RO * (1/d)) * (sv/448))
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, never frees and never synchronises except in
+ *     h3attn_check_status.  It keeps no state between calls other than a
+ *     per-device cache of kernel attributes.
+ *   - Element strides are in BF16 elements; the channel (d) stride is 1.
+ *     Base pointers must be 16-byte aligned and strides multiples of 8
+ *     elements (16-byte vector loads); the workspace must be 256-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously.  Argument errors are returned
+ *     synchronously and nothing is enqueued.  Errors found on the device (a
+ *     bounded wait that expired) are recorded in the workspace's status word
+ *     and returned by h3attn_check_status.
+ *   - Inputs are assumed finite; NaN or Inf inputs give undefined output.
+ *   - Output must not overlap the inputs or the workspace.
+ */
+#ifndef H3ATTN_H_
+#define H3ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define H3ATTN_VERSION 1
+#define H3ATTN_HEAD_DIM 128
+#define H3ATTN_Q_GROUP 32    /* Q tokens per INT8 scale ("per-warp" Q quantization) */
+#define H3ATTN_K_GROUP 64    /* K tokens per INT8 scale (one K64 epoch) */
+#define H3ATTN_TILE 128      /* Q rows and keys per tile of the attention kernel */
+
+typedef enum {
+  H3ATTN_OK = 0,
+  H3ATTN_ERR_INVALID_ARG = 1,  /* null pointer, size < 1, bad index */
+  H3ATTN_ERR_UNSUPPORTED = 2,  /* D != 128, or the current device is not sm_100 */
+  H3ATTN_ERR_ALIGNMENT = 3,    /* pointer or stride violates the alignment rules */
+  H3ATTN_ERR_WORKSPACE = 4,    /* workspace null, misaligned or smaller than needed */
+  H3ATTN_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed */
+  H3ATTN_ERR_TIMEOUT = 6       /* a device-side bounded wait expired (read via check_status) */
+} h3attn_status;
+
+/* A read-only BF16 tensor viewed as [B, T, H, D]; strides in elements, d stride 1. */
+typedef struct {
+  const void* data;
+  int64_t stride_b, stride_t, stride_h;
+} h3attn_bf16_view;
+
+/* A writable BF16 tensor viewed as [B, T, H, D]; strides in elements, d stride 1.
+ * The out-projection layout [B, T, H*D] is stride_b = T*H*D, stride_t = H*D, stride_h = D. */
+typedef struct {
+  void* data;
+  int64_t stride_b, stride_t, stride_h;
+} h3attn_bf16_out;
+
+/* Workspace fields, in the order h3attn_workspace_layout reports their byte offsets. */
+enum {
+  H3ATTN_WS_STATUS = 0, /* int32 status word (+ detail words), 256 bytes */
+  H3ATTN_WS_Q8,         /* int8  [B, H, Tq_pad, 128]   Tq_pad  = ceil(Tq/128)*128, rows >= Tq are 0 */
+  H3ATTN_WS_K8,         /* int8  [B, H, Tkv_pad, 128]  Tkv_pad = ceil(Tkv/128)*128, rows >= Tkv are 0 */
+  H3ATTN_WS_V8T,        /* e4m3  [B, H, 128, Tkv_pad]  V transposed (channel-major), columns >= Tkv are 0 */
+  H3ATTN_WS_SQ,         /* f32   [B, H, Tq_pad/32]     Q group scales (0 for groups past Tq) */
+  H3ATTN_WS_SK,         /* f32   [B, H, Tkv_pad/64]    K group scales (0 for groups past Tkv) */
+  H3ATTN_WS_KM,         /* f32   [B, H, 128]           K channel means */
+  H3ATTN_WS_SV,         /* f32   [B, H, 128]           V channel scales amax/448 */
+  H3ATTN_WS_KSUM,       /* f64   [B, H, ceil(Tkv/64), 128]  scratch: per-chunk K sums */
+  H3ATTN_WS_VMAX,       /* f32   [B, H, ceil(Tkv/64), 128]  scratch: per-chunk V absmax */
+  H3ATTN_WS_END,        /* total bytes */
+  H3ATTN_WS_NFIELDS
+};
+
+/* Bytes of workspace needed for (B, Tq, Tkv, H, D); 0 if the sizes are invalid. */
+size_t h3attn_workspace_bytes(int B, int Tq, int Tkv, int H, int D);
+
+/* Byte offsets of every workspace field (see the enum above) into offsets[H3ATTN_WS_NFIELDS]. */
+h3attn_status h3attn_workspace_layout(int B, int Tq, int Tkv, int H, int D,
+                                      int64_t offsets[H3ATTN_WS_NFIELDS]);
+
+/* K smoothing, Q/K INT8 and V FP8 quantization ("H3 Performance Roadmap", the
+ * Sage2 decomposition: K smoothing, Q/K INT8 quantization, V transpose and FP8
+ * quantization).  Reads q (Tq tokens) and k, v (Tkv tokens); writes every
+ * field of the workspace except the status word.  Three kernels:
+ * per-chunk statistics, their ordered reduction, one quantize pass. */
+h3attn_status h3attn_quantize_qkv(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                  const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* The fused attention mainloop on a workspace filled by h3attn_quantize_qkv with the
+ * same sizes: INT8 QK^T on the tensor cores into tensor memory, FP32 online softmax,
+ * FP8 P, FP8 PV with FP32 accumulation, final reciprocal, BF16 store of rows < Tq
+ * into `out`.  softmax_scale is usually 1/sqrt(D). */
+h3attn_status h3attn_attend(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H, int D,
+                            float softmax_scale, const h3attn_bf16_out* out, void* stream);
+
+/* Quantize + attend for self-attention (Tq == Tkv == T). */
+h3attn_status h3attn_forward(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                             const h3attn_bf16_view* v, int B, int T, int H, int D,
+                             float softmax_scale, const h3attn_bf16_out* out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Quantize + attend with separate query and key lengths. */
+h3attn_status h3attn_forward_ex(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                float softmax_scale, const h3attn_bf16_out* out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status recorded in the workspace
+ * (H3ATTN_OK or H3ATTN_ERR_TIMEOUT) and clears it.  ws must be at least 256 bytes. */
+h3attn_status h3attn_check_status(void* ws, void* stream);
+
+/* Parity export: the exact INT32 QK^T tile of (b, h, Q tile qt, key tile kt) as
+ * computed by the same tensor-core path the attention kernel uses, written as
+ * 128 x 128 row-major int32 to the device buffer out_dev. */
+h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H,
+                                     int D, int b, int h, int qt, int kt, int32_t* out_dev,
+                                     void* stream);
+
+/* Static description of a status code. */
+const char* h3attn_status_string(h3attn_status s);
+
+/* H3ATTN_VERSION of the loaded library. */
+int h3attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3ATTN_H_ */

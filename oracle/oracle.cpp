@@ -75,6 +75,16 @@ inline float e4m3_decode(uint8_t b) {
     return (float)(s ? -v : v);
 }
 
+// All 256 E4M3 values, decoded once by e4m3_decode (a lookup, not new arithmetic).
+struct E4M3Table {
+    float v[256];
+    E4M3Table() { for (int i = 0; i < 256; ++i) v[i] = e4m3_decode((uint8_t)i); }
+};
+const E4M3Table& e4m3_table() {
+    static const E4M3Table t;
+    return t;
+}
+
 // Round half to even of a non-negative double to an integer-valued double.
 inline double rne(double x) {
     double f = std::floor(x), r = x - f;
@@ -290,11 +300,12 @@ static void attend_row(const int8_t* q8, const int8_t* k8, const uint8_t* v8,
         }
         dsum = dsum * alpha + esum;
         // FP8 P times FP8 V, FP32 sums in ascending key order.
+        const float* dec = e4m3_table().v;
         for (int cc = 0; cc < D; ++cc) pv[cc] = 0.0f;
         for (int jj = 0; jj < n; ++jj) {
-            const float pj = e4m3_decode(p8[jj]);
+            const float pj = dec[p8[jj]];
             const uint8_t* vr = v8 + (bh * Tkv + j0 + jj) * D;
-            for (int cc = 0; cc < D; ++cc) pv[cc] += pj * e4m3_decode(vr[cc]);
+            for (int cc = 0; cc < D; ++cc) pv[cc] += pj * dec[vr[cc]];
         }
         for (int cc = 0; cc < D; ++cc) ro[cc] = ro[cc] * alpha + pv[cc];
         m = m_new;

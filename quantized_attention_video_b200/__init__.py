@@ -1,0 +1,195 @@
+"""Python binding of libh3attn.so (quantized dense self-attention for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of the shared library, reached through its C ABI with ctypes.  The
+functions carry the C names (``h3attn_forward`` ...) and take PyTorch CUDA
+tensors for device memory; PyTorch is used for nothing else.
+
+If the library has not been built this module raises on first use; there is
+no CPU fallback.  Build it with ``python -m quantized_attention_video_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libh3attn.so")
+
+HEAD_DIM = 128
+TILE = 128
+Q_GROUP = 32
+K_GROUP = 64
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+WS_FIELDS = ("status", "q8", "k8", "v8t", "sq", "sk", "km", "sv", "ksum", "vmax", "end")
+
+
+class H3AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {h3attn_status_string(status)} (status {status})")
+        self.status = status
+
+
+class _View(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("stride_b", ctypes.c_int64), ("stride_t", ctypes.c_int64),
+                ("stride_h", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libh3attn.so; raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m quantized_attention_video_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        I, P, S, F, I64 = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float, ctypes.c_int64
+        VP = ctypes.POINTER(_View)
+        L.h3attn_workspace_bytes.restype = S
+        L.h3attn_workspace_bytes.argtypes = [I] * 5
+        L.h3attn_workspace_layout.restype = I
+        L.h3attn_workspace_layout.argtypes = [I] * 5 + [ctypes.POINTER(I64)]
+        L.h3attn_quantize_qkv.restype = I
+        L.h3attn_quantize_qkv.argtypes = [VP, VP, VP] + [I] * 5 + [P, S, P]
+        L.h3attn_attend.restype = I
+        L.h3attn_attend.argtypes = [P, S] + [I] * 5 + [F, VP, P]
+        L.h3attn_forward.restype = I
+        L.h3attn_forward.argtypes = [VP, VP, VP] + [I] * 4 + [F, VP, P, S, P]
+        L.h3attn_forward_ex.restype = I
+        L.h3attn_forward_ex.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, P, S, P]
+        L.h3attn_check_status.restype = I
+        L.h3attn_check_status.argtypes = [P, P]
+        L.h3attn_debug_qk_scores.restype = I
+        L.h3attn_debug_qk_scores.argtypes = [P, S] + [I] * 9 + [P, P]
+        L.h3attn_status_string.restype = ctypes.c_char_p
+        L.h3attn_status_string.argtypes = [I]
+        L.h3attn_version.restype = I
+        L.h3attn_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------- marshalling --
+def _view(t) -> _View:
+    """[B, T, H, D] BF16 tensor (any strides, unit channel stride) -> view struct."""
+    if t.dim() != 4:
+        raise ValueError("expected a [B, T, H, D] tensor")
+    if t.stride(3) != 1:
+        raise ValueError("channel stride must be 1")
+    return _View(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr_bytes(ws):
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+def _check(st: int, where: str):
+    if st != OK:
+        raise H3AttnError(st, where)
+
+
+# -------------------------------------------------------------- C names ----
+def h3attn_status_string(status: int) -> str:
+    return lib().h3attn_status_string(status).decode()
+
+
+def h3attn_version() -> int:
+    return lib().h3attn_version()
+
+
+def h3attn_workspace_bytes(B: int, Tq: int, Tkv: int, H: int, D: int = HEAD_DIM) -> int:
+    return lib().h3attn_workspace_bytes(B, Tq, Tkv, H, D)
+
+
+def h3attn_workspace_layout(B: int, Tq: int, Tkv: int, H: int, D: int = HEAD_DIM) -> dict:
+    off = (ctypes.c_int64 * len(WS_FIELDS))()
+    _check(lib().h3attn_workspace_layout(B, Tq, Tkv, H, D, off), "h3attn_workspace_layout")
+    return dict(zip(WS_FIELDS, list(off)))
+
+
+def new_workspace(B: int, Tq: int, Tkv: int, H: int, device="cuda"):
+    """A uint8 device tensor of h3attn_workspace_bytes (PyTorch allocations are 512-byte aligned)."""
+    import torch
+    n = h3attn_workspace_bytes(B, Tq, Tkv, H)
+    if n == 0:
+        raise H3AttnError(ERR_INVALID_ARG, "h3attn_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def h3attn_quantize_qkv(q, k, v, ws, stream=None):
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(ws)
+    vq, vk, vv = _view(q), _view(k), _view(v)
+    _check(lib().h3attn_quantize_qkv(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H, D, wp, wb,
+                                     _stream(stream)), "h3attn_quantize_qkv")
+
+
+def h3attn_attend(ws, B: int, Tq: int, Tkv: int, H: int, softmax_scale: float, out, stream=None, D: int = HEAD_DIM):
+    wp, wb = _ptr_bytes(ws)
+    vo = _view(out)
+    _check(lib().h3attn_attend(wp, wb, B, Tq, Tkv, H, D, softmax_scale, ctypes.byref(vo), _stream(stream)),
+           "h3attn_attend")
+
+
+def h3attn_forward_ex(q, k, v, softmax_scale: float, out, ws, stream=None):
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(ws)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib().h3attn_forward_ex(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H, D,
+                                   softmax_scale, ctypes.byref(vo), wp, wb, _stream(stream)), "h3attn_forward_ex")
+
+
+def h3attn_forward(q, k, v, softmax_scale: float, out, ws, stream=None):
+    """Self-attention: q, k, v and out are [B, T, H, 128] BF16 views (out may be a view of [B, T, H*128])."""
+    B, T, H, D = q.shape
+    wp, wb = _ptr_bytes(ws)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib().h3attn_forward(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, T, H, D, softmax_scale,
+                                ctypes.byref(vo), wp, wb, _stream(stream)), "h3attn_forward")
+
+
+def h3attn_check_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib().h3attn_check_status(ws.data_ptr(), _stream(stream))
+
+
+def h3attn_debug_qk_scores(ws, B: int, Tq: int, Tkv: int, H: int, b: int, h: int, qt: int, kt: int, out,
+                           stream=None, D: int = HEAD_DIM):
+    """Exact INT32 QK^T tile (128 x 128) into the int32 device tensor `out`."""
+    wp, wb = _ptr_bytes(ws)
+    _check(lib().h3attn_debug_qk_scores(wp, wb, B, Tq, Tkv, H, D, b, h, qt, kt, out.data_ptr(), _stream(stream)),
+           "h3attn_debug_qk_scores")
+
+
+def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:
+    """Typed views of the workspace fields (for parity checks)."""
+    import torch
+    off = h3attn_workspace_layout(B, Tq, Tkv, H)
+    Tqp, Tkp = -(-Tq // TILE) * TILE, -(-Tkv // TILE) * TILE
+
+    def sl(name, n, dtype, shape):
+        nb = n * torch.tensor([], dtype=dtype).element_size()
+        return ws[off[name]:off[name] + nb].view(dtype).view(shape)
+
+    BH = B * H
+    return dict(
+        q8=sl("q8", BH * Tqp * 128, torch.int8, (B, H, Tqp, 128)),
+        k8=sl("k8", BH * Tkp * 128, torch.int8, (B, H, Tkp, 128)),
+        v8t=sl("v8t", BH * 128 * Tkp, torch.uint8, (B, H, 128, Tkp)),
+        sq=sl("sq", BH * (Tqp // Q_GROUP), torch.float32, (B, H, Tqp // Q_GROUP)),
+        sk=sl("sk", BH * (Tkp // K_GROUP), torch.float32, (B, H, Tkp // K_GROUP)),
+        km=sl("km", BH * 128, torch.float32, (B, H, 128)),
+        sv=sl("sv", BH * 128, torch.float32, (B, H, 128)),
+    )

@@ -1,0 +1,79 @@
+// Internal definitions shared by the host API and the kernels of libh3attn.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/h3attn.h"
+
+namespace h3 {
+
+constexpr int kD = H3ATTN_HEAD_DIM;     // head dimension (fixed)
+constexpr int kTile = H3ATTN_TILE;      // Q rows / keys per attention tile
+constexpr int kQGroup = H3ATTN_Q_GROUP; // Q tokens per scale
+constexpr int kKGroup = H3ATTN_K_GROUP; // K tokens per scale
+constexpr int kChunk = 64;              // tokens per K-mean / V-absmax partial
+
+struct Shape {
+  int B, Tq, Tkv, H;
+  int64_t Tq_pad, Tkv_pad;  // multiples of kTile
+  int64_t nchunk;           // ceil(Tkv / kChunk)
+};
+
+struct Layout {
+  int64_t off[H3ATTN_WS_NFIELDS];
+};
+
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+inline Shape make_shape(int B, int Tq, int Tkv, int H) {
+  Shape s;
+  s.B = B; s.Tq = Tq; s.Tkv = Tkv; s.H = H;
+  s.Tq_pad = round_up(Tq, kTile);
+  s.Tkv_pad = round_up(Tkv, kTile);
+  s.nchunk = (Tkv + kChunk - 1) / kChunk;
+  return s;
+}
+
+inline Layout make_layout(const Shape& s) {
+  const int64_t BH = (int64_t)s.B * s.H;
+  int64_t sz[H3ATTN_WS_NFIELDS] = {};
+  sz[H3ATTN_WS_STATUS] = 256;
+  sz[H3ATTN_WS_Q8] = BH * s.Tq_pad * kD;
+  sz[H3ATTN_WS_K8] = BH * s.Tkv_pad * kD;
+  sz[H3ATTN_WS_V8T] = BH * kD * s.Tkv_pad;
+  sz[H3ATTN_WS_SQ] = BH * (s.Tq_pad / kQGroup) * 4;
+  sz[H3ATTN_WS_SK] = BH * (s.Tkv_pad / kKGroup) * 4;
+  sz[H3ATTN_WS_KM] = BH * kD * 4;
+  sz[H3ATTN_WS_SV] = BH * kD * 4;
+  sz[H3ATTN_WS_KSUM] = BH * s.nchunk * kD * 8;
+  sz[H3ATTN_WS_VMAX] = BH * s.nchunk * kD * 4;
+  Layout L;
+  int64_t o = 0;
+  for (int f = 0; f < H3ATTN_WS_END; ++f) {
+    L.off[f] = o;
+    o = round_up(o + sz[f], 1024);
+  }
+  L.off[H3ATTN_WS_END] = o;
+  return L;
+}
+
+// Device-side status words at the start of the workspace.
+struct DevStatus {
+  int code;    // h3attn_status of the first failure, 0 if none
+  int detail;  // which wait expired (kernel-defined id)
+  int block;   // linear block index that recorded it
+  int pad[61];
+};
+
+// Kernel launchers (defined in quantize.cu / attention.cu).
+cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
+                            const Shape& s, const Layout& L, char* ws, cudaStream_t st);
+
+struct TmapSet;  // opaque; attention.cu
+cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
+                             const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why);
+cudaError_t launch_debug_qk(const char* ws, const Shape& s, const Layout& L, int b, int h, int qt, int kt,
+                            int32_t* out, cudaStream_t st, h3attn_status* why);
+
+}  // namespace h3

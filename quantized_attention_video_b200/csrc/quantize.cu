@@ -1,0 +1,301 @@
+// Preparation kernels of the quantized attention ("H3 Performance Roadmap",
+// the Sage2 decomposition: K smoothing, Q/K INT8 quantization, V transpose and
+// FP8 quantization; Phase 4 item 2: keep the per-warp INT8 Q/K and FP8 V policy).
+//
+//   stats_kernel    : one pass over K and V. Per (b, h, 64-token chunk, channel):
+//                     FP64 sum of K in token order, FP32 absmax of V.
+//   finalize_kernel : per (b, h, channel): K mean = (sum of chunk sums in chunk
+//                     order) / Tkv, rounded to FP32; V absmax and scale amax/448.
+//   quantize_kernel : one pass over Q, K, V in 128-token slabs. INT8 Q per
+//                     32-token group, INT8 (K - mean) per 64-token group, FP8 E4M3
+//                     V per channel written transposed (channel-major), zero
+//                     padding up to the 128-token tile multiple.
+//
+// All loads are 16-byte vectors of 8 BF16 channels; 16 threads cover one
+// 128-channel row, so a warp reads two contiguous 256-byte rows per load.
+#include <cuda_bf16.h>
+
+#include "h3attn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace h3 {
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// ------------------------------------------------------------------ stats ----
+// Thread (unit, sub): unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice.
+__global__ void __launch_bounds__(256) stats_kernel(const uint16_t* __restrict__ k, int64_t ksb, int64_t kst,
+                                                    int64_t ksh, const uint16_t* __restrict__ v, int64_t vsb,
+                                                    int64_t vst, int64_t vsh, int H, int Tkv, int64_t nchunk,
+                                                    int64_t nunits, double* __restrict__ ksum,
+                                                    float* __restrict__ vmax) {
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t unit = g >> 4;
+  const int sub = (int)(g & 15);
+  if (unit >= nunits) return;
+  const int64_t chunk = unit % nchunk, bh = unit / nchunk;
+  const int64_t h = bh % H, b = bh / H;
+  const int t0 = (int)(chunk * kChunk);
+  const int t1 = min(Tkv, t0 + kChunk);
+  const uint16_t* kp = k + b * ksb + h * ksh + sub * 8;
+  const uint16_t* vp = v + b * vsb + h * vsh + sub * 8;
+  double acc[8];
+  float vm[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { acc[e] = 0.0; vm[e] = 0.0f; }
+#pragma unroll 4
+  for (int t = t0; t < t1; ++t) {
+    float kf[8], vf[8];
+    unpack8(ldg16(kp + (int64_t)t * kst), kf);
+    unpack8(ldg16(vp + (int64_t)t * vst), vf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      acc[e] = __dadd_rn(acc[e], (double)kf[e]);
+      vm[e] = fmaxf(vm[e], fabsf(vf[e]));
+    }
+  }
+  double* ko = ksum + unit * kD + sub * 8;
+  float* vo = vmax + unit * kD + sub * 8;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { ko[e] = acc[e]; vo[e] = vm[e]; }
+}
+
+// --------------------------------------------------------------- finalize ----
+// One block of 128 threads per (b, h); thread = channel.  After it runs, chunk
+// row 0 of the V-absmax scratch holds the channel absmax over all keys.  It
+// also clears the workspace status word, so each quantize call starts clean.
+__global__ void __launch_bounds__(128) finalize_kernel(const double* __restrict__ ksum, float* __restrict__ vmax,
+                                                       int64_t nchunk, int Tkv, float* __restrict__ km,
+                                                       float* __restrict__ sv, DevStatus* status) {
+  const int64_t bh = blockIdx.x;
+  const int c = threadIdx.x;
+  if (bh == 0 && c == 0) {
+    status->code = 0;
+    status->detail = 0;
+    status->block = 0;
+  }
+  const double* kp = ksum + bh * nchunk * kD + c;
+  float* vp = vmax + bh * nchunk * kD + c;
+  double s = 0.0;
+  float m = 0.0f;
+  for (int64_t ch = 0; ch < nchunk; ++ch) {
+    s = __dadd_rn(s, kp[ch * kD]);
+    m = fmaxf(m, vp[ch * kD]);
+  }
+  km[bh * kD + c] = __double2float_rn(__ddiv_rn(s, (double)Tkv));
+  sv[bh * kD + c] = __fdiv_rn(m, 448.0f);
+  vp[0] = m;
+}
+
+// --------------------------------------------------------------- quantize ----
+__device__ __forceinline__ int8_t q_i8(float x, float inv) {
+  int r = __float2int_rn(__fmul_rn(x, inv));
+  r = max(-127, min(127, r));
+  return (int8_t)r;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+  return x;
+}
+
+// Thread (c16 = tid & 15, rq = tid >> 4) owns channels [8*c16, 8*c16+8) of the
+// 8 consecutive slab rows [8*rq, 8*rq+8).  Warp w covers slab rows [16w, 16w+16).
+__global__ void __launch_bounds__(256) quantize_kernel(
+    const uint16_t* __restrict__ q, int64_t qsb, int64_t qst, int64_t qsh,
+    const uint16_t* __restrict__ k, int64_t ksb, int64_t kst, int64_t ksh,
+    const uint16_t* __restrict__ v, int64_t vsb, int64_t vst, int64_t vsh,
+    int H, int Tq, int Tkv, int64_t Tq_pad, int64_t Tkv_pad, int64_t nchunk,
+    const float* __restrict__ km, const float* __restrict__ vmax,
+    int8_t* __restrict__ q8, float* __restrict__ sq, int8_t* __restrict__ k8, float* __restrict__ sk,
+    uint8_t* __restrict__ v8t) {
+  __shared__ float red[8];
+  __shared__ float gmax[4];
+  __shared__ __align__(16) uint8_t vt[kD * kTile];  // [channel][token], 16-byte chunks XOR-swizzled
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c16 = tid & 15, rq = tid >> 4;
+  const int64_t t0 = (int64_t)blockIdx.x * kTile;
+  const int64_t h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = b * H + h;
+
+  // ---------------------------------------------------------------- Q ----
+  if (t0 < Tq_pad) {
+    float x[8][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t t = t0 + 8 * rq + r;
+      if (t < Tq) {
+        unpack8(ldg16(q + b * qsb + t * qst + h * qsh + c16 * 8), x[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[r][e] = 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[r][e]));
+    }
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    if (tid < 4) {
+      const float a = fmaxf(red[2 * tid], red[2 * tid + 1]);
+      gmax[tid] = a;
+      sq[bh * (Tq_pad / kQGroup) + t0 / kQGroup + tid] = __fdiv_rn(a, 127.0f);
+    }
+    __syncthreads();
+    const float a = gmax[rq >> 2];
+    const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t t = t0 + 8 * rq + r;
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w0 |= (uint32_t)(uint8_t)q_i8(x[r][e], inv) << (8 * e);
+        w1 |= (uint32_t)(uint8_t)q_i8(x[r][e + 4], inv) << (8 * e);
+      }
+      *reinterpret_cast<uint2*>(q8 + (bh * Tq_pad + t) * kD + c16 * 8) = make_uint2(w0, w1);
+    }
+    __syncthreads();
+  }
+
+  if (t0 >= Tkv_pad) return;
+  // ---------------------------------------------------------------- K ----
+  {
+    float kmv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kmv[e] = km[bh * kD + c16 * 8 + e];
+    float x[8][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t t = t0 + 8 * rq + r;
+      if (t < Tkv) {
+        unpack8(ldg16(k + b * ksb + t * kst + h * ksh + c16 * 8), x[r]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], kmv[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[r][e] = 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[r][e]));
+    }
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    if (tid < 2) {
+      const float a = fmaxf(fmaxf(red[4 * tid], red[4 * tid + 1]), fmaxf(red[4 * tid + 2], red[4 * tid + 3]));
+      gmax[tid] = a;
+      sk[bh * (Tkv_pad / kKGroup) + t0 / kKGroup + tid] = __fdiv_rn(a, 127.0f);
+    }
+    __syncthreads();
+    const float a = gmax[rq >> 3];
+    const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t t = t0 + 8 * rq + r;
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w0 |= (uint32_t)(uint8_t)q_i8(x[r][e], inv) << (8 * e);
+        w1 |= (uint32_t)(uint8_t)q_i8(x[r][e + 4], inv) << (8 * e);
+      }
+      *reinterpret_cast<uint2*>(k8 + (bh * Tkv_pad + t) * kD + c16 * 8) = make_uint2(w0, w1);
+    }
+  }
+  // ---------------------------------------------------------------- V ----
+  {
+    float inv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float a = vmax[bh * nchunk * kD + c16 * 8 + e];
+      inv[e] = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+    }
+    uint8_t w[8][8];  // [channel e][row r]
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t t = t0 + 8 * rq + r;
+      float x[8];
+      if (t < Tkv) {
+        unpack8(ldg16(v + b * vsb + t * vst + h * vsh + c16 * 8), x);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const uint32_t p = cvt_e4m3x2(__fmul_rn(x[e], inv[e]), __fmul_rn(x[e + 1], inv[e + 1]));
+        w[e][r] = (uint8_t)(p & 0xFF);
+        w[e + 1][r] = (uint8_t)(p >> 8);
+      }
+    }
+    // rows [8rq, 8rq+8) of channel c are bytes [8rq, 8rq+8) of smem row c; the
+    // 16-byte chunk index is XORed with (c >> 3) & 7 to spread banks.
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c16 * 8 + e;
+      const int chunk = (rq >> 1) ^ ((c >> 3) & 7);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        lo |= (uint32_t)w[e][r] << (8 * r);
+        hi |= (uint32_t)w[e][r + 4] << (8 * r);
+      }
+      *reinterpret_cast<uint2*>(vt + c * kTile + chunk * 16 + (rq & 1) * 8) = make_uint2(lo, hi);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int vec = tid + 256 * j;
+      const int c = vec >> 3, part = vec & 7;
+      const int chunk = part ^ ((c >> 3) & 7);
+      const uint4 val = *reinterpret_cast<const uint4*>(vt + c * kTile + chunk * 16);
+      *reinterpret_cast<uint4*>(v8t + (bh * kD + c) * Tkv_pad + t0 + part * 16) = val;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
+                            const Shape& s, const Layout& L, char* ws, cudaStream_t st) {
+  auto* ksum = reinterpret_cast<double*>(ws + L.off[H3ATTN_WS_KSUM]);
+  auto* vmax = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_VMAX]);
+  auto* km = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_KM]);
+  auto* sv = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SV]);
+  const int64_t nunits = (int64_t)s.B * s.H * s.nchunk;
+  const int64_t threads = nunits * 16;
+  stats_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint16_t*>(k.data), k.stride_b, k.stride_t, k.stride_h,
+      static_cast<const uint16_t*>(v.data), v.stride_b, v.stride_t, v.stride_h, s.H, s.Tkv, s.nchunk, nunits,
+      ksum, vmax);
+  finalize_kernel<<<(unsigned)(s.B * s.H), 128, 0, st>>>(ksum, vmax, s.nchunk, s.Tkv, km, sv,
+                                                        reinterpret_cast<DevStatus*>(ws + L.off[H3ATTN_WS_STATUS]));
+  const int64_t slabs = (s.Tq_pad > s.Tkv_pad ? s.Tq_pad : s.Tkv_pad) / kTile;
+  dim3 grid((unsigned)slabs, (unsigned)s.H, (unsigned)s.B);
+  quantize_kernel<<<grid, 256, 0, st>>>(
+      static_cast<const uint16_t*>(q.data), q.stride_b, q.stride_t, q.stride_h,
+      static_cast<const uint16_t*>(k.data), k.stride_b, k.stride_t, k.stride_h,
+      static_cast<const uint16_t*>(v.data), v.stride_b, v.stride_t, v.stride_h, s.H, s.Tq, s.Tkv, s.Tq_pad,
+      s.Tkv_pad, s.nchunk, km, vmax, reinterpret_cast<int8_t*>(ws + L.off[H3ATTN_WS_Q8]),
+      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SQ]), reinterpret_cast<int8_t*>(ws + L.off[H3ATTN_WS_K8]),
+      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SK]), reinterpret_cast<uint8_t*>(ws + L.off[H3ATTN_WS_V8T]));
+  return cudaGetLastError();
+}
+
+}  // namespace h3

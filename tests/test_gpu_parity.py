@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bar (per the numerical policy of "H3 Performance Roadmap", Phase 4, and the
+checkpoints of "Phase 2B Aligned Numerical Prototype", Exactness):
+  * INT8 Q/K words, FP8 V words, every scale and the K means: bit-exact;
+  * INT32 QK^T scores: bit-exact (through the debug export, same MMA path);
+  * BF16 output: max-abs <= 1e-2 and relative L2 <= 2e-3 against the oracle run
+    with the kernel's 128-key softmax epoch.
+Inputs are the seeded synthetic workloads of the synth module.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import quantized_attention_video_b200 as h3
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+REL_L2 = 2e-3
+EPOCH = 128  # the kernel's key tile = its online-softmax epoch
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_attention_video_b200 import build
+    build.build()
+    h3.lib()  # raises loudly if the library is missing
+
+
+def upload(x: dict, w: synth.Workload):
+    """Device BF16 views for q, k, v (and the packed buffer when the workload is packed)."""
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+    if w.packed:
+        buf = dev(x["packed"])
+        return {"buf": buf, "q": buf[:, :, 0], "k": buf[:, :, 1], "v": buf[:, :, 2]}
+    return {n: dev(x[n]) for n in ("q", "k", "v")}
+
+
+def new_out(w: synth.Workload):
+    if w.packed:
+        o = torch.empty(w.B, w.Tq, w.H * w.D, dtype=torch.bfloat16, device="cuda")
+        return o, o.view(w.B, w.Tq, w.H, w.D)
+    o = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    return o, o
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    t = t.contiguous().cpu()
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def f32_bits(a: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.int32)
+
+
+def check_quantized(ws, z, w):
+    B, Tq, Tkv, H = w.B, w.Tq, w.Tkv, w.H
+    v = h3.workspace_views(ws, B, Tq, Tkv, H)
+    q8, k8, v8t = bits(v["q8"]), bits(v["k8"]), bits(v["v8t"])
+    assert np.array_equal(q8[:, :, :Tq], z["q8"]), "q8"
+    assert not q8[:, :, Tq:].any()
+    assert np.array_equal(k8[:, :, :Tkv], z["k8"]), "k8"
+    assert not k8[:, :, Tkv:].any()
+    assert np.array_equal(v8t[:, :, :, :Tkv].transpose(0, 1, 3, 2), z["v8"]), "v8"
+    assert not v8t[:, :, :, Tkv:].any()
+    nq, nk = z["sq"].shape[-1], z["sk"].shape[-1]
+    sq, sk = bits(v["sq"]), bits(v["sk"])
+    assert np.array_equal(sq[:, :, :nq], f32_bits(z["sq"])), "sq"
+    assert not sq[:, :, nq:].any()
+    assert np.array_equal(sk[:, :, :nk], f32_bits(z["sk"])), "sk"
+    assert not sk[:, :, nk:].any()
+    assert np.array_equal(bits(v["km"]), f32_bits(z["km"])), "km"
+    assert np.array_equal(bits(v["sv"]), f32_bits(z["sv"])), "sv"
+
+
+def compare_out(got: np.ndarray, ref: np.ndarray, what: str):
+    g = oracle.bf16_decode(got).astype(np.float64)
+    r = oracle.bf16_decode(ref).astype(np.float64)
+    assert np.isfinite(g).all(), what
+    err = np.abs(g - r)
+    rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+    assert err.max() <= MAX_ABS, f"{what}: max-abs {err.max():.3e}"
+    assert rel <= REL_L2, f"{what}: rel-L2 {rel:.3e}"
+    return err.max(), rel
+
+
+def sample_rows(w: synth.Workload, tiles_per_head: int, seed: int):
+    """(b, h, i) rows: the first and last (ragged) Q tile of every head plus random tiles."""
+    rng = np.random.default_rng(seed)
+    ntile = -(-w.Tq // 128)
+    rows = []
+    for b in range(w.B):
+        for h in range(w.H):
+            tiles = {0, ntile - 1} | set(rng.integers(0, ntile, size=tiles_per_head).tolist())
+            for t in sorted(tiles):
+                for i in range(t * 128, min(w.Tq, t * 128 + 128)):
+                    rows.append((b, h, i))
+    return np.array(rows, dtype=np.int32)
+
+
+def run_forward(w, d):
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    out, out4 = new_out(w)
+    if w.Tq == w.Tkv:
+        h3.h3attn_forward(d["q"], d["k"], d["v"], w.scale, out4, ws)
+    else:
+        h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, out4, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    return ws, out, out4
+
+
+# ---------------------------------------------------------------- configs ----
+FULL = ["fixed_q128_kv192", "selfattn_h8_t4096"]
+SAMPLED = {"ragged_h16_t9453": 3, "h3_t37810_h32": 1, "h3_packed_b2_t37810": 0}
+
+
+@pytest.mark.parametrize("name", FULL + list(SAMPLED))
+def test_workload_parity(name):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    z = oracle.quantize(x["q"], x["k"], x["v"])
+    d = upload(x, w)
+    ws, out, out4 = run_forward(w, d)
+    check_quantized(ws, z, w)
+    got = bits(out4)  # [B, T, H, D]
+    if name in FULL:
+        ref = oracle.attend_all(z, w.scale, EPOCH)
+        compare_out(got, ref, name)
+    else:
+        rows = sample_rows(w, SAMPLED[name], seed=w.seed)
+        ref, _, _ = oracle.attend_rows(z, w.scale, EPOCH, rows)
+        compare_out(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, name)
+    if w.packed:
+        # the output is the token-major [B, T, H*D] buffer itself
+        assert out.shape == (w.B, w.Tq, w.H * w.D) and out.is_contiguous()
+
+
+@pytest.mark.parametrize("name", FULL + list(SAMPLED))
+def test_qk_scores_bit_exact(name):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    z = oracle.quantize(x["q"], x["k"], x["v"])
+    d = upload(x, w)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    h3.h3attn_quantize_qkv(d["q"], d["k"], d["v"], ws)
+    nq, nk = -(-w.Tq // 128), -(-w.Tkv // 128)
+    rng = np.random.default_rng(7)
+    tiles = {(0, 0, 0, 0), (w.B - 1, w.H - 1, nq - 1, nk - 1)}
+    while len(tiles) < min(16, w.B * w.H * nq * nk):
+        tiles.add((int(rng.integers(w.B)), int(rng.integers(w.H)), int(rng.integers(nq)), int(rng.integers(nk))))
+    buf = torch.empty(128, 128, dtype=torch.int32, device="cuda")
+    for (b, h, qt, kt) in sorted(tiles):
+        h3.h3attn_debug_qk_scores(ws, w.B, w.Tq, w.Tkv, w.H, b, h, qt, kt, buf)
+        g = buf.cpu().numpy()
+        ni, nj = min(128, w.Tq - qt * 128), min(128, w.Tkv - kt * 128)
+        ref = oracle.scores(z, b, h, qt * 128, ni, kt * 128, nj)
+        assert np.array_equal(g[:ni, :nj], ref), (b, h, qt, kt)
+        # padded rows / keys are zero words, so their scores are exactly 0
+        assert not g[ni:].any() and not g[:, nj:].any()
+    assert h3.h3attn_check_status(ws) == h3.OK
+
+
+# ------------------------------------------------------------- edge cases ----
+EDGE = [(1, 1, 1, 1), (1, 1, 200, 1), (1, 200, 1, 1), (1, 127, 129, 2), (2, 129, 127, 1), (1, 255, 256, 1),
+        (1, 257, 300, 3), (3, 64, 64, 2), (1, 384, 640, 1), (1, 130, 1000, 2)]
+
+
+@pytest.mark.parametrize("B,Tq,Tkv,H", EDGE)
+def test_edge_shapes(B, Tq, Tkv, H):
+    w = synth.Workload(f"edge_{B}_{Tq}_{Tkv}_{H}", B, Tq, Tkv, H, 128, "normal", 1000 + Tq * 7 + Tkv)
+    x = synth.make_inputs(w)
+    z = oracle.quantize(x["q"], x["k"], x["v"])
+    d = upload(x, w)
+    ws, out, out4 = run_forward(w, d)
+    check_quantized(ws, z, w)
+    compare_out(bits(out4), oracle.attend_all(z, w.scale, EPOCH), w.name)
+
+
+def test_degenerate_zero_inputs():
+    w = synth.Workload("zeros", 1, 200, 300, 2, 128, "normal", 5)
+    x = synth.make_inputs(w)
+    x["q"][:, :, 0] = 0          # head 0: all-zero Q -> uniform softmax
+    x["k"][:, :, 1] = 0          # head 1: all-zero K -> zero scores
+    x["v"][:, 50:, 1, :64] = 0   # some V channels zero after token 50
+    x["v"][:, :, 0, 100:] = 0    # V channels that are zero everywhere -> zero scale, zero output
+    z = oracle.quantize(x["q"], x["k"], x["v"])
+    d = upload(x, w)
+    ws, out, out4 = run_forward(w, d)
+    check_quantized(ws, z, w)
+    got = bits(out4)
+    compare_out(got, oracle.attend_all(z, w.scale, EPOCH), "zeros")
+    assert not got[:, :, 0, 100:].any()
+
+
+def test_output_strides_and_untouched_padding():
+    """Output written through a strided view; rows and channels outside it stay untouched."""
+    w = synth.Workload("strided_out", 1, 300, 300, 2, 128, "normal", 77)
+    x = synth.make_inputs(w)
+    z = oracle.quantize(x["q"], x["k"], x["v"])
+    d = upload(x, w)
+    big = torch.full((1, 300, 2, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    view = big[:, :, :, 64:192]
+    ws = h3.new_workspace(1, 300, 300, 2)
+    h3.h3attn_forward(d["q"], d["k"], d["v"], w.scale, view, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    compare_out(bits(view), oracle.attend_all(z, w.scale, EPOCH), "strided")
+    assert (big[:, :, :, :64] == 7.0).all() and (big[:, :, :, 192:] == 7.0).all()
+
+
+def test_repeated_launches_are_deterministic():
+    """The fixed shape relaunched many times gives the same output bytes (no hang, no race)."""
+    w = synth.WORKLOADS["fixed_q128_kv192"]
+    x = synth.make_inputs(w)
+    d = upload(x, w)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    out = torch.empty(1, 128, 1, 128, dtype=torch.bfloat16, device="cuda")
+    h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, out, ws)
+    first = bits(out).tobytes()
+    for _ in range(200):
+        h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, out, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    assert bits(out).tobytes() == first
