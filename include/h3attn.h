@@ -139,6 +139,25 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
                                      int D, int b, int h, int qt, int kt, int32_t* out_dev,
                                      void* stream);
 
+/* Size of the device array behind h3attn_forward_static (64 MiB). */
+#define H3ATTN_STATIC_WS_BYTES (64u << 20)
+
+/* Forward pass (quantize + attend, Tq and Tkv as in h3attn_forward_ex) for callers that
+ * cannot allocate device memory: a host that owns the device allocator and offers this
+ * library no way to request memory, or a runtime that forbids allocation after start-up.
+ * The pages have no counterpart; it is an interface addition of this library.
+ * Takes the inputs and the output only. The workspace is a file-scope device array of
+ * H3ATTN_STATIC_WS_BYTES that every GPU loading the library holds until exit; shapes
+ * whose h3attn_workspace_bytes exceeds it return H3ATTN_ERR_WORKSPACE. The first call
+ * on a device (with that device current) looks up the array's address; make that first
+ * call before any stream capture. Calls no cudaMalloc or cudaFree. All calls share the
+ * array, which keeps the last call's contents, so calls whose GPU work overlaps race on
+ * it; the caller must order them. Device-side wait timeouts are recorded in the array's
+ * status word, which this interface does not expose. */
+h3attn_status h3attn_forward_static(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                    const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                    float softmax_scale, const h3attn_bf16_out* out, void* stream);
+
 /* Static description of a status code. */
 const char* h3attn_status_string(h3attn_status s);
 

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.h3attn_forward.argtypes = [VP, VP, VP] + [I] * 4 + [F, VP, P, S, P]
         L.h3attn_forward_ex.restype = I
         L.h3attn_forward_ex.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, P, S, P]
+        L.h3attn_forward_static.restype = I
+        L.h3attn_forward_static.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, P]
         L.h3attn_check_status.restype = I
         L.h3attn_check_status.argtypes = [P, P]
         L.h3attn_debug_qk_scores.restype = I
@@ -158,6 +160,20 @@ def h3attn_forward(q, k, v, softmax_scale: float, out, ws, stream=None):
     vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
     _check(lib().h3attn_forward(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, T, H, D, softmax_scale,
                                 ctypes.byref(vo), wp, wb, _stream(stream)), "h3attn_forward")
+
+
+STATIC_WS_BYTES = 64 << 20
+
+
+def h3attn_forward_static(q, k, v, softmax_scale: float, out, stream=None):
+    """Forward pass without a caller workspace: the library's static 64 MiB device array
+    is used instead (for callers that cannot allocate device memory).  The first call on
+    a device should come before any stream capture; calls whose GPU work overlaps race."""
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib().h3attn_forward_static(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H, D,
+                                       softmax_scale, ctypes.byref(vo), _stream(stream)), "h3attn_forward_static")
 
 
 def h3attn_check_status(ws, stream=None) -> int:
