@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.h3attn_check_status.argtypes = [P, P]
         L.h3attn_debug_qk_scores.restype = I
         L.h3attn_debug_qk_scores.argtypes = [P, S] + [I] * 9 + [P, P]
+        L.h3attn_debug_attend_trace.restype = I
+        L.h3attn_debug_attend_trace.argtypes = [P, S] + [I] * 5 + [F, VP, I, P, P]
         L.h3attn_status_string.restype = ctypes.c_char_p
         L.h3attn_status_string.argtypes = [I]
         L.h3attn_version.restype = I
@@ -187,6 +189,23 @@ def h3attn_debug_qk_scores(ws, B: int, Tq: int, Tkv: int, H: int, b: int, h: int
     wp, wb = _ptr_bytes(ws)
     _check(lib().h3attn_debug_qk_scores(wp, wb, B, Tq, Tkv, H, D, b, h, qt, kt, out.data_ptr(), _stream(stream)),
            "h3attn_debug_qk_scores")
+
+
+TRACE_EVENTS = ("s_ready", "alpha", "p_done", "qk_issue", "pv_issue", "o_corrected", "k_full", "probs")
+
+
+def h3attn_debug_attend_trace(ws, B: int, Tq: int, Tkv: int, H: int, softmax_scale: float, out, trace_block: int,
+                              stream=None, D: int = HEAD_DIM):
+    """h3attn_attend with a clock64 timeline of one CTA; returns {event: int64 [2, nkv]} (0 = not recorded)."""
+    import torch
+    nkv = -(-Tkv // TILE)
+    tr = torch.zeros(len(TRACE_EVENTS) * 2 * nkv, dtype=torch.int64, device=out.device)
+    wp, wb = _ptr_bytes(ws)
+    vo = _view(out)
+    _check(lib().h3attn_debug_attend_trace(wp, wb, B, Tq, Tkv, H, D, softmax_scale, ctypes.byref(vo), trace_block,
+                                           tr.data_ptr(), _stream(stream)), "h3attn_debug_attend_trace")
+    t = tr.view(len(TRACE_EVENTS), 2, nkv).cpu()
+    return {name: t[i] for i, name in enumerate(TRACE_EVENTS)}
 
 
 def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:

@@ -171,6 +171,28 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
   return H3ATTN_OK;
 }
 
+h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H, int D,
+                                        float softmax_scale, const h3attn_bf16_out* out, int trace_block,
+                                        uint64_t* trace_dev, void* stream) {
+  H3_TRY(check_sizes(B, Tq, Tkv, H, D));
+  H3_TRY(check_out(out));
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return H3ATTN_ERR_INVALID_ARG;
+  if (trace_dev == nullptr) return H3ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(trace_dev) % 8 != 0) return H3ATTN_ERR_ALIGNMENT;
+  const Shape s = make_shape(B, Tq, Tkv, H);
+  const Layout L = make_layout(s);
+  const int64_t ctas = (s.Tq_pad / kTile) * (int64_t)H * B;
+  if (trace_block < 0 || trace_block >= ctas) return H3ATTN_ERR_INVALID_ARG;
+  H3_TRY(check_ws(ws, ws_bytes, L));
+  H3_TRY(check_device());
+  const float c_log2 = (float)((double)softmax_scale * kLog2e);
+  h3attn_status why = H3ATTN_OK;
+  if (launch_attention(static_cast<const char*>(ws), s, L, c_log2, *out, static_cast<cudaStream_t>(stream), &why,
+                       trace_dev, trace_block) != cudaSuccess)
+    return why != H3ATTN_OK ? why : H3ATTN_ERR_CUDA;
+  return H3ATTN_OK;
+}
+
 const char* h3attn_status_string(h3attn_status s) {
   switch (s) {
     case H3ATTN_OK: return "ok";

@@ -2,26 +2,33 @@
 // Phase 4: Dense Sage-Compatible Attention; numerical checkpoints of "Phase 2B
 // Aligned Numerical Prototype", Exactness).
 //
-// One CTA owns two 128-row Q tiles (A and B) of one (b, h) and streams all
-// 128-key K/V tiles past them.  Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K and V^T tiles into a
-//               3-stage shared-memory ring (separate K and V barriers).
-//   warp 1      tensor-memory allocator and single-thread MMA issuer:
-//               S = Q K^T  with tcgen05.mma kind::i8 (INT8 x INT8 -> S32),
-//               O += P V   with tcgen05.mma kind::f8f6f4 (E4M3, A = P read
-//               from tensor memory, F32 accumulate).
-//   warps 2-3   stage the per-channel output scales, then idle.
-//   warps 4-7   softmax + correction + epilogue for Q tile A,
-//   warps 8-11  the same for Q tile B.  Thread = one Q row (= one TMEM lane).
-// Tensor memory (512 columns): S_A [0,128) S_B [128,256) O_A [256,384)
-// O_B [384,512).  P (128 x 128 E4M3 = 32 columns) overwrites the first 32
-// columns of its S after the scores were read.  MMAs issued by one thread run
-// in order, so S of tile j+1 is written only after P of tile j was consumed.
-// The MMA order per key tile j keeps the tensor pipe busy while one softmax
-// warpgroup works: QK_A(j), PV_B(j-1), QK_B(j), PV_A(j).
+// One CTA owns one 128-row Q tile of one (b, h) and streams all 128-key K/V
+// tiles past it.  Warp roles (512 threads, four warpgroups):
+//   WG0  warp 0   TMA producer of the Q tile and the K tiles (4-stage ring).
+//        warp 2   TMA producer of the V^T tiles (4-stage ring), so K tiles
+//                 run ahead of V tiles by as much as the rings allow.
+//        warp 1   tensor-memory allocator and single-thread MMA issuer:
+//                 S = Q K^T  tcgen05.mma kind::i8 (INT8 x INT8 -> S32),
+//                 O += P V   tcgen05.mma kind::f8f6f4 (E4M3, A = P read from
+//                 tensor memory, F32 accumulate).
+//        warp 3   stages the per-channel output scales, then idles.
+//   WG1  softmax of the even key tiles (scores in S0)  } thread = one Q row.
+//   WG2  softmax of the odd key tiles (scores in S1)   } The running row max
+//        is handed from the warpgroup of tile j to that of tile j+1, so one
+//        warpgroup's max/exchange phase overlaps the other's exp2 phase.
+//   WG3  O correction (rescale by alpha when the running max moves) and the
+//        epilogue (final reciprocal, BF16 store).
+// Tensor memory (512 columns allocated): S0 [0,128) S1 [128,256) O [256,384)
+// P0 [384,416) P1 [416,448).  Scores of key tile j go to S(j%2) and its E4M3
+// probabilities (128 x 128 bytes = 32 columns) to P(j%2).  The softmax frees
+// S(j%2) as soon as it has read the scores, so QK(j+2) runs on the tensor
+// cores while the softmax of tile j is still computing; it writes P(j%2)
+// only after PV(j-2) has consumed the previous contents.
 //
-// Every wait is bounded: after the limit the waiter records H3ATTN_ERR_TIMEOUT
-// in the workspace status word, raises a CTA-wide abort flag, drains the
+// Every hand-off whose producer could otherwise run two phases ahead of its
+// consumer uses two barriers (indexed by key tile parity).  Every wait is
+// bounded: after the limit the waiter records H3ATTN_ERR_TIMEOUT in the
+// workspace status word, raises a CTA-wide abort flag, drains the
 // asynchronous work it issued and leaves; the tensor memory is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -35,42 +42,49 @@
 namespace h3 {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = 128 * 128;
-constexpr uint32_t kColSA = 0, kColSB = 128, kColOA = 256, kColOB = 384;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 416;
 constexpr uint32_t kIdescQK = idesc_i8_s32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // setmaxnreg split (registers per thread): control, correction, softmax warpgroups.
-constexpr int kRegsControl = 56, kRegsCorrection = 96, kRegsSoftmax = 176;
+constexpr int kRegsControl = 64, kRegsCorrection = 80, kRegsSoftmax = 176;
 constexpr int64_t kRegSplitTotal = 128 * (kRegsControl + kRegsCorrection + 2 * kRegsSoftmax);
 static_assert(kRegSplitTotal <= 65536, "register split exceeds the SM register file");
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 
 struct __align__(1024) AttnSmem {
-  uint8_t q[2][kTileBytes];
+  uint8_t q[kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2];
-  uint64_t a_full[2];   // softmax -> correction: alpha of the key tile published (one phase per tile)
-  uint64_t o_ready[2];  // correction -> MMA issuer: O rescaled for the key tile
-  uint64_t d_full[2];   // softmax -> correction: final row sum d published (one phase)
+  uint64_t s_full[2];   // MMA -> softmax: scores of key tile j in S(j%2)
+  uint64_t s_free[2];   // softmax -> MMA: scores of key tile j read, S(j%2) may be overwritten
+  uint64_t p_full[2];   // softmax -> MMA: P of key tile j in P(j%2)
+  uint64_t a_full[2];   // softmax -> correction: alpha of key tile j in alpha[j%2]
+  uint64_t m_full[2];   // softmax of tile j -> softmax of tile j+1: running max in mrow[j%2]
+  uint64_t o_ready[2];  // correction -> MMA: O rescaled for key tile j
+  uint64_t pv_done[2];  // MMA -> correction, softmax: PV of key tile j completed (P(j%2) free)
+  uint64_t o_full;      // MMA -> epilogue: the last PV completed
+  uint64_t d_full;      // softmax (both warpgroups) -> epilogue: partial row sums published
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  float svs[kD];
+  float sv[kD];
   float alpha[2][kTile];
-  float dsum[2][kTile];
+  float mrow[2][kTile];   // [key tile parity][row]: running max after that tile (log2 domain)
+  float dsum[2][kTile];   // [warpgroup][row]: sum of 448*p over its tiles, relative to mlast
+  float mlast[2][kTile];  // [warpgroup][row]: running max at its last tile
 };
 
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
-  kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaPA, kSiteMmaPB, kSiteMmaV,
-  kSiteSoftS, kSiteSoftO, kSiteMmaO, kSiteCorrA, kSiteCorrS, kSiteEpiO
+  kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
+  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrA, kSiteCorrPV, kSiteEpi
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
@@ -88,98 +102,64 @@ __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int quarter, u
 
 constexpr uint32_t kMagic = 0x4B400000u;  // bit pattern of 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;     // 1.5 * 2^23
+constexpr float kLog2_448 = 8.80735492205760410749f;
 
-// Maximum of 64 INT32 scores of one row (tile columns col0 ..); with kMasked,
-// columns >= valid (keys past Tkv) are ignored.  Eight independent chains.
-template <bool kMasked, int kCol0>
-__device__ __forceinline__ int rowmax64(const uint32_t (&s)[128], int valid) {
-  int m[8];
+// The 128 INT32 scores of a row become x = 1.5*2^23 + acc as FP32 bit patterns
+// (exact, |acc| < 2^22), in place; x is monotone in acc, so the row maxima of
+// the two 64-key halves (one K scale each) are taken on x.  With kMasked,
+// columns >= valid (keys past Tkv) become 0, below every x.
+template <bool kMasked>
+__device__ __forceinline__ void magic_and_max(uint32_t (&s)[128], int valid, float& xm0, float& xm1) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = INT_MIN;
-#pragma unroll
-  for (int e = 0; e < 64; ++e) {
-    int v = (int)s[kCol0 + e];
-    if (kMasked && kCol0 + e >= valid) v = INT_MIN;
-    m[e & 7] = max(m[e & 7], v);
+  for (int e = 0; e < 128; ++e) {
+    uint32_t v = s[e] + kMagic;
+    if (kMasked && e >= valid) v = 0u;
+    s[e] = v;
   }
-  return max(max(max(m[0], m[1]), max(m[2], m[3])), max(max(m[4], m[5]), max(m[6], m[7])));
+  float m[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m[c] = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 128; e += 2) {
+    const int c = ((e >> 1) & 3) + (e >= 64 ? 4 : 0);
+    m[c] = fmax3(m[c], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+  }
+  xm0 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  xm1 = fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// Probabilities of 64 scores of one row: t = float(acc) * f (float(acc) exact
-// through the 1.5*2^23 magic number, |acc| < 2^22), p = 2^(t - m) in FP32,
-// FP32 partial sums of p into acc2, E4M3 words of 448*p into w[0..15] (4 per word).
-template <bool kMasked, int kCol0>
-__device__ __forceinline__ void probs64(const uint32_t (&s)[128], int valid, float f, float m,
-                                        uint64_t (&acc2)[4], uint32_t (&w)[32]) {
+// Scaled probabilities of the 128 keys of a row: q = 2^((x - 1.5*2^23)*f - mq)
+// with mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
+// into acc2 and the E4M3 words of q into w (4 keys per word).
+template <bool kMasked>
+__device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
+                                         uint64_t (&acc2)[4], uint32_t (&w)[32]) {
   const uint64_t negC = f2_pack(-kMagicF, -kMagicF);
-  const uint64_t ff = f2_pack(f, f);
-  const uint64_t negm = f2_pack(-m, -m);
-  const uint64_t c448 = f2_pack(448.0f, 448.0f);
+  const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
+  const uint64_t negm = f2_pack(-mq, -mq);
 #pragma unroll
-  for (int e = 0; e < 64; e += 4) {
+  for (int e = 0; e < 128; e += 4) {
     uint32_t half[2];
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
-      const int i = kCol0 + e + 2 * hp;
-      const uint64_t x = f2_pack(__uint_as_float(s[i] + kMagic), __uint_as_float(s[i + 1] + kMagic));
-      const uint64_t u = f2_add(f2_mul(f2_add(x, negC), ff), negm);
+      const int i = e + 2 * hp;
+      const uint64_t a = f2_add(f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1])), negC);
+      const uint64_t u = f2_fma(a, i < 64 ? ff0 : ff1, negm);
       float u0, u1;
       f2_unpack(u, u0, u1);
-      float p0 = ex2_ftz(u0), p1 = ex2_ftz(u1);
+      float q0 = ex2_ftz(u0), q1 = ex2_ftz(u1);
       if (kMasked) {
-        if (i >= valid) p0 = 0.0f;
-        if (i + 1 >= valid) p1 = 0.0f;
+        if (i >= valid) q0 = 0.0f;
+        if (i + 1 >= valid) q1 = 0.0f;
       }
-      const uint64_t pp = f2_pack(p0, p1);
-      acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], pp);
-      float q0, q1;
-      f2_unpack(f2_mul(pp, c448), q0, q1);
+      acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(q0, q1));
       half[hp] = cvt_e4m3x2(q0, q1);
     }
-    w[(kCol0 + e) >> 2] = half[0] | (half[1] << 16);
+    w[e >> 2] = half[0] | (half[1] << 16);
   }
 }
 
-// One key tile of the online softmax for the row this thread owns: reads the
-// INT32 scores from tensor memory (tS), updates the running max m; publishes
-// alpha = 2^(m_old - m_new) to the correction warpgroup as soon as it is known
-// (alpha_slot, a_bar), then writes the 32 E4M3 probability words over the first
-// 32 score columns, hands them to the MMA issuer (p_bar) and updates the sum d.
-template <bool kMasked>
-__device__ __forceinline__ void softmax_tile(uint32_t tS, float f0, float f1, int valid, float& m, float& dsum,
-                                             float* alpha_slot, uint64_t* a_bar, uint64_t* p_bar) {
-  uint32_t pw[32];
-  uint64_t acc2[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
-  float m_new, alpha;
-  {
-    uint32_t sc[128];
-    tmem_ld64x2(tS, sc);
-    const int mi0 = rowmax64<kMasked, 0>(sc, valid);
-    const int mi1 = rowmax64<kMasked, 64>(sc, valid);
-    const float t0m = mi0 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mi0), f0);
-    const float t1m = mi1 == INT_MIN ? -INFINITY : __fmul_rn(__int2float_rn(mi1), f1);
-    m_new = fmaxf(m, fmaxf(t0m, t1m));
-    alpha = ex2_approx(__fsub_rn(m, m_new));
-    *alpha_slot = alpha;
-    mbar_arrive(a_bar);
-    probs64<kMasked, 0>(sc, valid, f0, m_new, acc2, pw);
-    probs64<kMasked, 64>(sc, valid, f1, m_new, acc2, pw);
-  }
-  tmem_st32(tS, pw);
-  tmem_wait_st();
-  tc_fence_before();
-  mbar_arrive(p_bar);
-  float a[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
-  const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-  dsum = __fadd_rn(__fmul_rn(dsum, alpha), es);
-  m = m_new;
-}
-
-// End of every role: all 384 threads meet, then warp 1 frees the tensor memory.
+// End of every role: all 512 threads meet, then warp 1 frees the tensor memory.
 __device__ __forceinline__ void attn_teardown(uint32_t tmem, bool owner) {
   tc_fence_before();
   __syncthreads();
@@ -188,6 +168,20 @@ __device__ __forceinline__ void attn_teardown(uint32_t tmem, bool owner) {
     tmem_dealloc(tmem, 512);
   }
 }
+
+// Timeline trace (debug export only): clock64() of per-key-tile events of one CTA,
+// trace[(event * 2 + slot) * nkv + j]; slot = key half for the softmax events, 0 otherwise.
+enum : int {
+  kEvSReady = 0,   // softmax warp: scores of key tile j ready (after the wait)
+  kEvAlpha = 1,    // softmax warp: row maximum exchanged, alpha known
+  kEvPDone = 2,    // softmax warp: probabilities stored, MMA issuer signalled
+  kEvQK = 3,       // MMA issuer: QK of key tile j issued
+  kEvPV = 4,       // MMA issuer: P and O ready, PV of key tile j issued
+  kEvCorr = 5,     // correction warp: O rescaled (or skipped), MMA issuer signalled
+  kEvKFull = 6,    // MMA issuer: K tile j landed in shared memory
+  kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed (before the P store)
+  kNumEvents = 8
+};
 
 struct AttnParams {
   const float* sq;   // [B,H,Tq_pad/32]
@@ -199,8 +193,11 @@ struct AttnParams {
   int64_t Tq_pad, Tkv_pad;
   float c_log2;      // float(softmax_scale * log2(e))
   DevStatus* status;
+  uint64_t* trace;   // timeline trace buffer (traced instantiation only)
+  int trace_block;   // linear block index that records the trace
 };
 
+template <bool kTrace>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -210,11 +207,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2, quarter = warp & 3;
   const int64_t h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
-  const int qt0 = 2 * blockIdx.x;                       // Q tile index of tile A
-  const bool has_b = (int64_t)(qt0 + 1) * kTile < p.Tq;  // tile B holds at least one row
-  const int ntiles = has_b ? 2 : 1;
+  const int qt = blockIdx.x;  // Q tile index
   const int nkv = (p.Tkv + kTile - 1) / kTile;
   volatile int* abort = &sm.abort;
+  const bool tracing =
+      kTrace && (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) == p.trace_block;
+  auto trace = [&](int ev, int slot, int j) {
+    if (kTrace && tracing) p.trace[(int64_t)(ev * 2 + slot) * nkv + j] = clock_now();
+  };
 
   // ------------------------------------------------------------ set-up ----
   if (warp == 0 && lane == 0) {
@@ -225,14 +225,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.p_full[t], kTile);
-      mbar_init(&sm.o_full[t], 1);
-      mbar_init(&sm.a_full[t], kTile);
-      mbar_init(&sm.o_ready[t], kTile);
-      mbar_init(&sm.d_full[t], kTile);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_free[i], kTile);
+      mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.p_full[i], kTile);
+      mbar_init(&sm.a_full[i], kTile);
+      mbar_init(&sm.m_full[i], kTile);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.o_ready[i], kTile);
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.d_full, 2 * kTile);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     mbar_fence_init();
@@ -241,57 +244,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 2 || warp == 3) {
-    for (int c = threadIdx.x - 64; c < kD; c += 64) sm.svs[c] = __fdiv_rn(p.sv[bh * kD + c], 448.0f);
+  if (warp == 3) {
+    for (int c = lane; c < kD; c += 32) sm.sv[c] = p.sv[bh * kD + c];
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  // Register split of the 512 x 128 launch budget: control warpgroup 56,
-  // correction warpgroup 96, each softmax warpgroup 176:
-  // 128*56 + 128*96 + 256*176 = 64512 <= 65536.  The host checks that the
+  // Register split of the 512 x 128 launch budget: control warpgroup 64,
+  // correction warpgroup 80, each softmax warpgroup 176:
+  // 128*64 + 128*80 + 256*176 = 63488 <= 65536.  The host checks that the
   // kernel was built with 128 registers per thread before launching.
   if (wg == 0) {
     regs_dealloc<kRegsControl>();
     if (warp == 0) {
-      // ---------------------------------------------------- TMA producer ----
+      // ---------------------------------------------- TMA producer: Q, K ----
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        const int qrow = (int)(bh * p.Tq_pad + (int64_t)qt0 * kTile);
-        mbar_arrive_expect_tx(&sm.q_full, has_b ? 2 * kTileBytes : kTileBytes);
-        tma_load_2d(sm.q[0], &tm_q, &sm.q_full, 0, qrow);
-        if (has_b) tma_load_2d(sm.q[1], &tm_q, &sm.q_full, 0, qrow + kTile);
+        mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+        tma_load_2d(sm.q, &tm_q, &sm.q_full, 0, (int)(bh * p.Tq_pad + (int64_t)qt * kTile));
         const int krow = (int)(bh * p.Tkv_pad);
-        const int vrow = (int)(bh * kD);
-        int issued_k = 0, issued_v = 0;
+        int issued = 0;
         for (int j = 0; j < nkv; ++j) {
           const int s = j % kStages;
-          const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-          if (!mbar_wait(&sm.k_empty[s], ph ^ 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.k_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdKEmpty, abort);
             break;
           }
           mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
           tma_load_2d(sm.k[s], &tm_k, &sm.k_full[s], 0, krow + j * kTile);
-          issued_k = j + 1;
-          if (!mbar_wait(&sm.v_empty[s], ph ^ 1u, abort, kWaitLimitNs)) {
+          issued = j + 1;
+        }
+        if (*abort) {
+          // let every copy this thread started land before the CTA can exit
+          mbar_wait(&sm.q_full, 0, nullptr, kDrainLimitNs);
+          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+            mbar_wait(&sm.k_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, kDrainLimitNs);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ------------------------------------------------- TMA producer: V ----
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_v);
+        const int vrow = (int)(bh * kD);
+        int issued = 0;
+        for (int j = 0; j < nkv; ++j) {
+          const int s = j % kStages;
+          if (!mbar_wait(&sm.v_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdVEmpty, abort);
             break;
           }
           mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
           tma_load_2d(sm.v[s], &tm_v, &sm.v_full[s], j * kTile, vrow);
-          issued_v = j + 1;
+          issued = j + 1;
         }
         if (*abort) {
-          // let every copy this thread started land before the CTA can exit
-          mbar_wait(&sm.q_full, 0, nullptr, kDrainLimitNs);
-          for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
-            mbar_wait(&sm.k_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, kDrainLimitNs);
-          for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
+          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
             mbar_wait(&sm.v_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, kDrainLimitNs);
         }
       }
@@ -302,64 +313,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = mbar_wait(&sm.q_full, 0, abort, kWaitLimitNs);
         if (!ok) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaQ, abort);
         tc_fence_after();
-        const uint64_t dq0 = sdesc_k_sw128(smem_u32(sm.q[0]));
-        const uint64_t dq1 = sdesc_k_sw128(smem_u32(sm.q[1]));
-        // PV of tile t for key tile jj once its P and its rescaled O are ready
-        auto pv = [&](int t, int jj) -> bool {
-          if (!mbar_wait(&sm.p_full[t], (uint32_t)jj & 1u, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, t ? kSiteMmaPB : kSiteMmaPA, abort);
-            return false;
-          }
-          if (!mbar_wait(&sm.o_ready[t], (uint32_t)jj & 1u, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
+        const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q));
+        // S(jj%2) = Q K(jj)^T
+        auto qk = [&](int jj) -> bool {
+          const int s = jj % kStages;
+          if (!mbar_wait(&sm.k_full[s], (uint32_t)(jj / kStages) & 1u, abort, kWaitLimitNs)) {
+            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
             return false;
           }
           tc_fence_after();
-          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.v[jj % kStages]));
-          const uint32_t o_col = t ? kColOB : kColOA, s_col = t ? kColSB : kColSA;
+          trace(kEvKFull, 0, jj);
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s]));
+          const uint32_t s_col = (jj & 1) ? kColS1 : kColS0;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts(tmem + o_col, tmem + s_col + 8 * kk, dv + 2 * kk, kIdescPV, jj > 0 || kk > 0);
+          for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + s_col, dq + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
+          mma_commit(&sm.s_full[jj & 1]);
+          mma_commit(&sm.k_empty[s]);
+          trace(kEvQK, 0, jj);
           return true;
         };
+        if (ok) ok = qk(0);
+        if (ok && nkv > 1) ok = qk(1);
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStages;
-          const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-          if (!mbar_wait(&sm.k_full[s], ph, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
+          if (j + 2 < nkv) {
+            // S(j%2) is free once the softmax of tile j has read its scores
+            if (!mbar_wait(&sm.s_free[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
+              record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaS, abort);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (!(ok = qk(j + 2))) break;
+          }
+          if (!mbar_wait(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
+            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s]));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + kColSA, dq0 + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
-          mma_commit(&sm.s_full[0]);
-          if (has_b) {
-            if (j > 0) {
-              if (!(ok = pv(1, j - 1))) break;
-              mma_commit(&sm.v_empty[(j - 1) % kStages]);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + kColSB, dq1 + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
-            mma_commit(&sm.s_full[1]);
+          if (!mbar_wait(&sm.o_ready[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
+            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
+            ok = false;
+            break;
           }
-          mma_commit(&sm.k_empty[s]);
-          if (!mbar_wait(&sm.v_full[s], ph, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStages) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaV, abort);
             ok = false;
             break;
           }
-          if (!(ok = pv(0, j))) break;
-          if (!has_b) mma_commit(&sm.v_empty[s]);
-          if (j == nkv - 1) mma_commit(&sm.o_full[0]);
+          tc_fence_after();
+          trace(kEvPV, 0, j);
+          const uint64_t dv = sdesc_k_sw128(smem_u32(sm.v[s]));
+          const uint32_t p_col = (j & 1) ? kColP1 : kColP0;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts(tmem + kColO, tmem + p_col + 8 * kk, dv + 2 * kk, kIdescPV, j > 0 || kk > 0);
+          mma_commit(&sm.pv_done[j & 1]);
+          mma_commit(&sm.v_empty[s]);
         }
-        if (ok && has_b) {
-          if ((ok = pv(1, nkv - 1))) {
-            mma_commit(&sm.v_empty[(nkv - 1) % kStages]);
-            mma_commit(&sm.o_full[1]);
-          }
-        }
+        if (ok) mma_commit(&sm.o_full);
         // wait until every MMA this thread issued has completed
         mma_commit(&sm.drain);
         mbar_wait(&sm.drain, 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
@@ -374,52 +386,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (wg == 3) {
     // -------------------------------------------- correction + epilogue ----
     regs_dealloc<kRegsCorrection>();
+    const uint32_t tO = tmem_lane_addr(tmem, quarter, kColO);
     bool ok = true;
-    for (int j = 0; ok && j < nkv; ++j) {
-      for (int t = 0; t < ntiles; ++t) {
-        ok = mbar_wait(&sm.a_full[t], (uint32_t)j & 1u, abort, kWaitLimitNs) &&
-             mbar_wait(&sm.s_full[t], (uint32_t)j & 1u, abort, kWaitLimitNs);
+    for (int j = 0; j < nkv; ++j) {
+      ok = mbar_wait(&sm.a_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) {
+        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrA, abort);
+        break;
+      }
+      const float alpha = sm.alpha[j & 1][row];
+      if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+        // O holds the sum over key tiles < j once the PV of tile j-1 has completed
+        ok = mbar_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort, kWaitLimitNs);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
-          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrA, abort);
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
           break;
         }
         tc_fence_after();
-        const float alpha = sm.alpha[t][row];
-        // O holds the sum over key tiles < j and the PV of tile j-1 has completed
-        if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-          const uint32_t tO = tmem_lane_addr(tmem, quarter, t ? kColOB : kColOA);
-          const uint64_t aa = f2_pack(alpha, alpha);
+        const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * ch, o);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * ch, o);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
-              o[e] = __float_as_uint(lo);
-              o[e + 1] = __float_as_uint(hi);
-            }
-            tmem_st32(tO + 32 * ch, o);
+          for (int e = 0; e < 32; e += 2) {
+            float lo, hi;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
+            o[e] = __float_as_uint(lo);
+            o[e + 1] = __float_as_uint(hi);
           }
-          tmem_wait_st();
+          tmem_st32(tO + 32 * ch, o);
         }
-        tc_fence_before();
-        mbar_arrive(&sm.o_ready[t]);
+        tmem_wait_st();
       }
+      tc_fence_before();
+      mbar_arrive(&sm.o_ready[j & 1]);
+      if (quarter == 0 && lane == 0) trace(kEvCorr, 0, j);
     }
-    for (int t = 0; ok && t < ntiles; ++t) {
-      ok = mbar_wait(&sm.d_full[t], 0, abort, kWaitLimitNs) && mbar_wait(&sm.o_full[t], 0, abort, kWaitLimitNs);
+    if (ok) {
+      ok = mbar_wait(&sm.d_full, 0, abort, kWaitLimitNs) && mbar_wait(&sm.o_full, 0, abort, kWaitLimitNs);
       ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) {
-        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteEpiO, abort);
-        break;
-      }
+      if (!ok && lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteEpi, abort);
+    }
+    if (ok) {
       tc_fence_after();
-      const float r = __frcp_rn(sm.dsum[t][row]);
-      const int64_t grow = (int64_t)(qt0 + t) * kTile + row;
-      const uint32_t tO = tmem_lane_addr(tmem, quarter, t ? kColOB : kColOA);
+      // d = sum over tiles of 448*p relative to the final max, from the two warpgroups
+      const float m0 = sm.mlast[0][row], m1 = sm.mlast[1][row];
+      const float mf = fmaxf(m0, m1);
+      const float d = __fadd_rn(__fmul_rn(sm.dsum[0][row], ex2_approx(__fsub_rn(m0, mf))),
+                                __fmul_rn(sm.dsum[1][row], ex2_approx(__fsub_rn(m1, mf))));
+      const float r = __frcp_rn(d);
+      const int64_t grow = (int64_t)qt * kTile + row;
       __nv_bfloat16* orow = p.out + b * p.out_sb + grow * p.out_st + h * p.out_sh;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -432,8 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int c0 = 32 * ch + e + 2 * u;
-              const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u]), r), sm.svs[c0]);
-              const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u + 1]), r), sm.svs[c0 + 1]);
+              const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u]), r), sm.sv[c0]);
+              const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u + 1]), r), sm.sv[c0 + 1]);
               const __nv_bfloat162 pr2 = __floats2bfloat162_rn(y0, y1);
               w[u] = *reinterpret_cast<const uint32_t*>(&pr2);
             }
@@ -448,38 +467,100 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // -------------------------------------------------------- softmax ----
   regs_alloc<kRegsSoftmax>();
-  const int t = wg - 1;  // 0 = tile A, 1 = tile B
-  if (t < ntiles) {
-    const int qt = qt0 + t;
+  const int par = wg - 1;  // this warpgroup owns key tiles j with j % 2 == par (scores in S(par))
+  {
     const float sqi = p.sq[bh * (p.Tq_pad / kQGroup) + (int64_t)qt * (kTile / kQGroup) + quarter];
     const float* skh = p.sk + bh * (p.Tkv_pad / kKGroup);
-    const uint32_t tS = tmem_lane_addr(tmem, quarter, t ? kColSB : kColSA);
-    float m = -INFINITY, dsum = 0.0f;
-    float sk0 = __ldg(skh + 0), sk1 = __ldg(skh + 1);
+    const uint32_t tS = tmem_lane_addr(tmem, quarter, par ? kColS1 : kColS0);
+    const uint32_t tP = tmem_lane_addr(tmem, quarter, par ? kColP1 : kColP0);
+    float m_w = -INFINITY, d_w = 0.0f;  // running max at this warpgroup's previous tile, its sum
+    float sk0 = 0.0f, sk1 = 0.0f;
+    if (par < nkv) {
+      sk0 = __ldg(skh + 2 * par);
+      sk1 = __ldg(skh + 2 * par + 1);
+    }
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = par; j < nkv; j += 2) {
       const float f0 = __fmul_rn(__fmul_rn(sqi, sk0), p.c_log2);
       const float f1 = __fmul_rn(__fmul_rn(sqi, sk1), p.c_log2);
-      if (j + 1 < nkv) {
-        sk0 = __ldg(skh + 2 * (j + 1));
-        sk1 = __ldg(skh + 2 * (j + 1) + 1);
+      if (j + 2 < nkv) {
+        sk0 = __ldg(skh + 2 * (j + 2));
+        sk1 = __ldg(skh + 2 * (j + 2) + 1);
       }
-      ok = mbar_wait(&sm.s_full[t], (uint32_t)j & 1u, abort, kWaitLimitNs);
+      ok = mbar_wait(&sm.s_full[par], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
         if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
         break;
       }
       tc_fence_after();
+      const bool tr = kTrace && tracing && quarter == 0 && lane == 0;
+      if (tr) trace(kEvSReady, par, j);
       const int valid = min(kTile, p.Tkv - j * kTile);
+      uint32_t x[128];
+      tmem_ld64x2(tS, x);
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[par]);
+      float xm0, xm1;
       if (valid < kTile)
-        softmax_tile<true>(tS, f0, f1, valid, m, dsum, &sm.alpha[t][row], &sm.a_full[t], &sm.p_full[t]);
+        magic_and_max<true>(x, valid, xm0, xm1);
       else
-        softmax_tile<false>(tS, f0, f1, valid, m, dsum, &sm.alpha[t][row], &sm.a_full[t], &sm.p_full[t]);
+        magic_and_max<false>(x, valid, xm0, xm1);
+      const float t0m = valid > 0 ? __fmul_rn(__fsub_rn(xm0, kMagicF), f0) : -INFINITY;
+      const float t1m = valid > 64 ? __fmul_rn(__fsub_rn(xm1, kMagicF), f1) : -INFINITY;
+      // running max after tile j-1, from the other warpgroup
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        ok = mbar_wait(&sm.m_full[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort, kWaitLimitNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftM, abort);
+          break;
+        }
+        m_prev = sm.mrow[(j - 1) & 1][row];
+      }
+      const float m_j = fmaxf(m_prev, fmaxf(t0m, t1m));
+      sm.mrow[j & 1][row] = m_j;
+      mbar_arrive(&sm.m_full[j & 1]);
+      sm.alpha[j & 1][row] = ex2_approx(__fsub_rn(m_prev, m_j));
+      mbar_arrive(&sm.a_full[j & 1]);
+      if (tr) trace(kEvAlpha, par, j);
+      uint32_t pw[32];
+      uint64_t acc2[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
+      const float mq = __fsub_rn(m_j, kLog2_448);
+      if (valid < kTile)
+        probs128<true>(x, valid, f0, f1, mq, acc2, pw);
+      else
+        probs128<false>(x, valid, f0, f1, mq, acc2, pw);
+      if (tr) trace(kEvProbs, par, j);
+      if (j >= 2) {
+        // P(j%2) still feeds PV(j-2) until that MMA has completed
+        ok = mbar_wait(&sm.pv_done[par], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftPV, abort);
+          break;
+        }
+        tc_fence_after();
+      }
+      tmem_st32(tP, pw);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[par]);
+      if (tr) trace(kEvPDone, par, j);
+      float a[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
+      const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+      d_w = __fadd_rn(__fmul_rn(d_w, ex2_approx(__fsub_rn(m_w, m_j))), es);
+      m_w = m_j;
     }
     if (ok) {
-      sm.dsum[t][row] = dsum;
-      mbar_arrive(&sm.d_full[t]);
+      sm.dsum[par][row] = d_w;
+      sm.mlast[par][row] = m_w;
+      mbar_arrive(&sm.d_full);
     }
   }
   attn_teardown(tmem, false);
@@ -596,15 +677,19 @@ cudaError_t ensure_attrs() {
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(mu);
   if (dev < 32 && (done_mask >> dev) & 1) return cudaSuccess;
-  e = cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
+  e = cudaFuncSetAttribute(attn_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(debug_qk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDebugSmemBytes);
   if (e != cudaSuccess) return e;
   // The warpgroup register split (setmaxnreg) needs the full launch budget.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_sm100_kernel);
-  if (e != cudaSuccess) return e;
-  if ((int64_t)fa.numRegs * kThreads < kRegSplitTotal) return cudaErrorInvalidConfiguration;
+  for (int traced = 0; traced < 2; ++traced) {
+    e = cudaFuncGetAttributes(&fa, traced ? (const void*)attn_sm100_kernel<true> : (const void*)attn_sm100_kernel<false>);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * kThreads < kRegSplitTotal) return cudaErrorInvalidConfiguration;
+  }
   if (dev < 32) done_mask |= 1 << dev;
   return cudaSuccess;
 }
@@ -612,7 +697,8 @@ cudaError_t ensure_attrs() {
 }  // namespace
 
 cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
-                             const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why) {
+                             const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why, uint64_t* trace,
+                             int trace_block) {
   *why = H3ATTN_OK;
   cudaError_t e = ensure_attrs();
   if (e != cudaSuccess) return e;
@@ -639,9 +725,13 @@ cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, fl
   p.Tkv_pad = s.Tkv_pad;
   p.c_log2 = c_log2;
   p.status = reinterpret_cast<DevStatus*>(const_cast<char*>(ws) + L.off[H3ATTN_WS_STATUS]);
-  const unsigned pairs = (unsigned)((s.Tq_pad / kTile + 1) / 2);
-  dim3 grid(pairs, (unsigned)s.H, (unsigned)s.B);
-  attn_sm100_kernel<<<grid, kThreads, kAttnSmemBytes, st>>>(tq, tk, tv, p);
+  p.trace = trace;
+  p.trace_block = trace_block;
+  dim3 grid((unsigned)(s.Tq_pad / kTile), (unsigned)s.H, (unsigned)s.B);
+  if (trace != nullptr)
+    attn_sm100_kernel<true><<<grid, kThreads, kAttnSmemBytes, st>>>(tq, tk, tv, p);
+  else
+    attn_sm100_kernel<false><<<grid, kThreads, kAttnSmemBytes, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -16,6 +16,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+__device__ __forceinline__ uint64_t clock_now() {
+  uint64_t c;
+  asm volatile("mov.u64 %0, %clock64;" : "=l"(c));
+  return c;
+}
+
 // ------------------------------------------------------------- mbarrier ----
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -304,6 +310,17 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+// Maximum of three FP32 values.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // Warpgroup register reallocation (all four warps of a warpgroup execute it).
 template <uint32_t kRegs>
 __device__ __forceinline__ void regs_dealloc() {
@@ -335,10 +352,10 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
 // Instruction descriptor: D format in bits 4-5 (1 = F32, 2 = S32), A format in
 // 7-9, B format in 10-12 (8-bit integer: 1 = signed; FP8: 0 = E4M3), both
 // operands K-major (bits 15, 16 = 0), N >> 3 in 17-22, M >> 4 in 24-28.
-constexpr uint32_t idesc_i8_s32(int M, int N) {
+__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
