@@ -7,11 +7,15 @@
 //   WG0  warp 0   TMA producer of the Q tile and the K tiles (4-stage ring).
 //        warp 2   TMA producer of the V^T tiles (4-stage ring), so K tiles
 //                 run ahead of V tiles by as much as the rings allow.
-//        warp 1   tensor-memory allocator and single-thread MMA issuer:
-//                 S = Q K^T  tcgen05.mma kind::i8 (INT8 x INT8 -> S32),
+//        warp 1   tensor-memory allocator and QK issuer (one thread):
+//                 S = Q K^T  tcgen05.mma kind::i8 (INT8 x INT8 -> S32).
+//        warp 3   PV issuer (one thread):
 //                 O += P V   tcgen05.mma kind::f8f6f4 (E4M3, A = P read from
 //                 tensor memory, F32 accumulate).
-//        warp 3   stages the per-channel output scales, then idles.
+//                 A tcgen05.mma issue blocks for about its execution time, so
+//                 the two products have their own issuing threads and neither
+//                 waits behind the other's dependencies.  Their MMAs touch
+//                 disjoint tensor memory; every true dependency is a barrier.
 //   WG1  softmax of the even key tiles (scores in S0)  } thread = one Q row.
 //   WG2  softmax of the odd key tiles (scores in S1)   } The running row max
 //        is handed from the warpgroup of tile j to that of tile j+1, so one
@@ -36,6 +40,7 @@
 #include <climits>
 #include <mutex>
 
+#include "exp2_poly.h"
 #include "h3attn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -50,7 +55,7 @@ constexpr uint32_t kIdescQK = idesc_i8_s32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // setmaxnreg split (registers per thread): control, correction, softmax warpgroups.
-constexpr int kRegsControl = 64, kRegsCorrection = 80, kRegsSoftmax = 176;
+constexpr int kRegsControl = 64, kRegsCorrection = 56, kRegsSoftmax = 192;
 constexpr int64_t kRegSplitTotal = 128 * (kRegsControl + kRegsCorrection + 2 * kRegsSoftmax);
 static_assert(kRegSplitTotal <= 65536, "register split exceeds the SM register file");
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
@@ -66,12 +71,13 @@ struct __align__(1024) AttnSmem {
   uint64_t s_free[2];   // softmax -> MMA: scores of key tile j read, S(j%2) may be overwritten
   uint64_t p_full[2];   // softmax -> MMA: P of key tile j in P(j%2)
   uint64_t a_full[2];   // softmax -> correction: alpha of key tile j in alpha[j%2]
+  uint64_t a_free[2];   // correction -> softmax: alpha of key tile j read, alpha[j%2] may be rewritten
   uint64_t m_full[2];   // softmax of tile j -> softmax of tile j+1: running max in mrow[j%2]
   uint64_t o_ready[2];  // correction -> MMA: O rescaled for key tile j
   uint64_t pv_done[2];  // MMA -> correction, softmax: PV of key tile j completed (P(j%2) free)
   uint64_t o_full;      // MMA -> epilogue: the last PV completed
   uint64_t d_full;      // softmax (both warpgroups) -> epilogue: partial row sums published
-  uint64_t drain;
+  uint64_t drain[2];  // QK issuer, PV issuer: all own MMAs completed
   uint32_t tmem_base;
   int abort;
   float sv[kD];
@@ -84,7 +90,7 @@ struct __align__(1024) AttnSmem {
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
-  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrA, kSiteCorrPV, kSiteEpi
+  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteSoftA, kSiteCorrA, kSiteCorrPV, kSiteEpi
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
@@ -128,9 +134,37 @@ __device__ __forceinline__ void magic_and_max(uint32_t (&s)[128], int valid, flo
   xm1 = fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
+// 2^u for a pair of arguments on the FMA pipe instead of the MUFU unit
+// (Cody-Waite range reduction and the polynomial of exp2_poly.h): n = rint(u)
+// through the 1.5*2^23 magic number, r = u - n exactly, 2^r by Horner in
+// packed FP32, then 2^n added into the exponent field.  u is clamped to
+// >= -125 so that the result stays normal (below that 2^u is < 2^-125 and
+// rounds to the E4M3 zero like the hardware exp2 does).
+__device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) {
+  float u0, u1;
+  f2_unpack(u, u0, u1);
+  const uint64_t uc = f2_pack(fmaxf(u0, -125.0f), fmaxf(u1, -125.0f));
+  const uint64_t y = f2_add(uc, f2_pack(kMagicF, kMagicF));   // 1.5*2^23 + n
+  const uint64_t n = f2_add(y, f2_pack(-kMagicF, -kMagicF));  // n
+  const uint64_t r = f2_fma(n, f2_pack(-1.0f, -1.0f), uc);    // u - n
+  uint64_t pp = f2_fma(f2_pack(kExp2C5, kExp2C5), r, f2_pack(kExp2C4, kExp2C4));
+  pp = f2_fma(pp, r, f2_pack(kExp2C3, kExp2C3));
+  pp = f2_fma(pp, r, f2_pack(kExp2C2, kExp2C2));
+  pp = f2_fma(pp, r, f2_pack(kExp2C1, kExp2C1));
+  pp = f2_fma(pp, r, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, y0, y1;
+  f2_unpack(pp, p0, p1);
+  f2_unpack(y, y0, y1);
+  // bits(y) << 23 == n << 23 (mod 2^32): the magic number's low 9 bits are zero
+  q0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
+  q1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
+}
+
 // Scaled probabilities of the 128 keys of a row: q = 2^((x - 1.5*2^23)*f - mq)
 // with mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
-// into acc2 and the E4M3 words of q into w (4 keys per word).
+// into acc2 and the E4M3 words of q into w (4 keys per word).  One key pair in
+// four takes its exp2 from the FMA pipe (exp2_fma_pair), the rest from MUFU,
+// which balances the two units.
 template <bool kMasked>
 __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
                                          uint64_t (&acc2)[4], uint32_t (&w)[32]) {
@@ -145,9 +179,15 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
       const int i = e + 2 * hp;
       const uint64_t a = f2_add(f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1])), negC);
       const uint64_t u = f2_fma(a, i < 64 ? ff0 : ff1, negm);
-      float u0, u1;
-      f2_unpack(u, u0, u1);
-      float q0 = ex2_ftz(u0), q1 = ex2_ftz(u1);
+      float q0, q1;
+      if (((i >> 1) & 3) == 3) {
+        exp2_fma_pair(u, q0, q1);
+      } else {
+        float u0, u1;
+        f2_unpack(u, u0, u1);
+        q0 = ex2_ftz(u0);
+        q1 = ex2_ftz(u1);
+      }
       if (kMasked) {
         if (i >= valid) q0 = 0.0f;
         if (i + 1 >= valid) q1 = 0.0f;
@@ -180,7 +220,9 @@ enum : int {
   kEvCorr = 5,     // correction warp: O rescaled (or skipped), MMA issuer signalled
   kEvKFull = 6,    // MMA issuer: K tile j landed in shared memory
   kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed (before the P store)
-  kNumEvents = 8
+  kEvPVDone = 8,   // MMA issuer: PV of key tile j issued and committed
+  kEvSFree = 9,    // MMA issuer: scores of key tile j released by the softmax (QK(j+2) may start)
+  kNumEvents = 10
 };
 
 struct AttnParams {
@@ -231,12 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.p_full[i], kTile);
       mbar_init(&sm.a_full[i], kTile);
+      mbar_init(&sm.a_free[i], kTile);
       mbar_init(&sm.m_full[i], kTile);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&sm.o_ready[i], kTile);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.d_full, 2 * kTile);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     sm.abort = 0;
     mbar_fence_init();
   }
@@ -244,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 3) {
+  if (warp == 4) {
     for (int c = lane; c < kD; c += 32) sm.sv[c] = p.sv[bh * kD + c];
   }
   tc_fence_before();
@@ -253,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   // Register split of the 512 x 128 launch budget: control warpgroup 64,
-  // correction warpgroup 80, each softmax warpgroup 176:
-  // 128*64 + 128*80 + 256*176 = 63488 <= 65536.  The host checks that the
+  // correction warpgroup 56, each softmax warpgroup 192:
+  // 128*64 + 128*56 + 256*192 = 64512 <= 65536.  The host checks that the
   // kernel was built with 128 registers per thread before launching.
   if (wg == 0) {
     regs_dealloc<kRegsControl>();
@@ -308,44 +352,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else if (warp == 1) {
-      // ------------------------------------------------------ MMA issuer ----
+      // ------------------------------------------------ QK issuer ----
       if (lane == 0) {
         bool ok = mbar_wait(&sm.q_full, 0, abort, kWaitLimitNs);
         if (!ok) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaQ, abort);
         tc_fence_after();
         const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q));
-        // S(jj%2) = Q K(jj)^T
-        auto qk = [&](int jj) -> bool {
-          const int s = jj % kStages;
-          if (!mbar_wait(&sm.k_full[s], (uint32_t)(jj / kStages) & 1u, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
-            return false;
-          }
-          tc_fence_after();
-          trace(kEvKFull, 0, jj);
-          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s]));
-          const uint32_t s_col = (jj & 1) ? kColS1 : kColS0;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + s_col, dq + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
-          mma_commit(&sm.s_full[jj & 1]);
-          mma_commit(&sm.k_empty[s]);
-          trace(kEvQK, 0, jj);
-          return true;
-        };
-        if (ok) ok = qk(0);
-        if (ok && nkv > 1) ok = qk(1);
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStages;
-          if (j + 2 < nkv) {
-            // S(j%2) is free once the softmax of tile j has read its scores
-            if (!mbar_wait(&sm.s_free[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
+          if (j >= 2) {
+            // S(j%2) is free once the softmax of tile j-2 has read its scores
+            if (!mbar_wait(&sm.s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs)) {
               record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaS, abort);
               ok = false;
               break;
             }
             tc_fence_after();
-            if (!(ok = qk(j + 2))) break;
+            trace(kEvSFree, 0, j - 2);
           }
+          if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, abort, kWaitLimitNs)) {
+            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          trace(kEvKFull, 0, j);
+          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s]));
+          const uint32_t s_col = (j & 1) ? kColS1 : kColS0;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + s_col, dq + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
+          mma_commit(&sm.s_full[j & 1]);
+          mma_commit(&sm.k_empty[s]);
+          trace(kEvQK, 0, j);
+        }
+        // wait until every MMA this thread issued has completed
+        mma_commit(&sm.drain[0]);
+        mbar_wait(&sm.drain[0], 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
+      }
+      __syncwarp();
+    } else if (warp == 3) {
+      // ------------------------------------------------ PV issuer ----
+      if (lane == 0) {
+        bool ok = true;
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int s = j % kStages;
           if (!mbar_wait(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
             ok = false;
@@ -370,11 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f8_ts(tmem + kColO, tmem + p_col + 8 * kk, dv + 2 * kk, kIdescPV, j > 0 || kk > 0);
           mma_commit(&sm.pv_done[j & 1]);
           mma_commit(&sm.v_empty[s]);
+          trace(kEvPVDone, 0, j);
         }
         if (ok) mma_commit(&sm.o_full);
-        // wait until every MMA this thread issued has completed
-        mma_commit(&sm.drain);
-        mbar_wait(&sm.drain, 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
+        mma_commit(&sm.drain[1]);
+        mbar_wait(&sm.drain[1], 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
       }
       __syncwarp();
     }
@@ -396,30 +446,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const float alpha = sm.alpha[j & 1][row];
-      if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-        // O holds the sum over key tiles < j once the PV of tile j-1 has completed
+      mbar_arrive(&sm.a_free[j & 1]);
+      if (j > 0) {
+        // O holds the sum over key tiles < j once the PV of tile j-1 has completed.  The
+        // wait also keeps this warpgroup from running two tiles ahead of the PV issuer.
         ok = mbar_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort, kWaitLimitNs);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
           break;
         }
-        tc_fence_after();
-        const uint64_t aa = f2_pack(alpha, alpha);
+        if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+          tc_fence_after();
+          const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * ch, o);
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * ch, o);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float lo, hi;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
-            o[e] = __float_as_uint(lo);
-            o[e + 1] = __float_as_uint(hi);
+            for (int e = 0; e < 32; e += 2) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
+              o[e] = __float_as_uint(lo);
+              o[e + 1] = __float_as_uint(hi);
+            }
+            tmem_st32(tO + 32 * ch, o);
           }
-          tmem_st32(tO + 32 * ch, o);
+          tmem_wait_st();
         }
-        tmem_wait_st();
       }
       tc_fence_before();
       mbar_arrive(&sm.o_ready[j & 1]);
@@ -522,6 +576,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_j = fmaxf(m_prev, fmaxf(t0m, t1m));
       sm.mrow[j & 1][row] = m_j;
       mbar_arrive(&sm.m_full[j & 1]);
+      if (j >= 2) {
+        // the correction warpgroup has read alpha of tile j-2 from this slot
+        ok = mbar_wait(&sm.a_free[par], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftA, abort);
+          break;
+        }
+      }
       sm.alpha[j & 1][row] = ex2_approx(__fsub_rn(m_prev, m_j));
       mbar_arrive(&sm.a_full[j & 1]);
       if (tr) trace(kEvAlpha, par, j);
