@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-sample-rows", type=int, default=48)
+    ap.add_argument("--cpu-sample-rows", type=int, default=0,
+                    help="query rows of head 0 timed on the CPU oracle (0 = all Tq rows of that head)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
@@ -78,16 +79,21 @@ def cpu_oracle_sample(w: synth.Workload, rows_per_head: int, x=None):
     z = oracle.quantize(q, k, v)
     t_quant = time.perf_counter() - t0
     rng = np.random.default_rng(0)
-    rows = np.stack([np.zeros(rows_per_head, int), np.zeros(rows_per_head, int),
-                     np.sort(rng.choice(w.Tq, rows_per_head, replace=False))], axis=1)
+    if rows_per_head <= 0 or rows_per_head >= w.Tq:
+        rows_per_head = w.Tq
+        picked = np.arange(w.Tq)
+    else:
+        picked = np.sort(rng.choice(w.Tq, rows_per_head, replace=False))
+    rows = np.stack([np.zeros(rows_per_head, int), np.zeros(rows_per_head, int), picked], axis=1)
     t0 = time.perf_counter()
     oracle.attend_rows(z, w.scale, 128, rows)
     t_rows = time.perf_counter() - t0
     # the quantize pass is shared by all Tq rows of the head; charge its share
     secs = t_rows + t_quant * rows_per_head / w.Tq
     ops = 4.0 * rows_per_head * w.Tkv * w.D
+    what = "all" if rows_per_head == w.Tq else f"{rows_per_head} random"
     text = (f"{w.name}: quantize of 1 of {w.B * w.H} heads ({t_quant:.2f} s, charged pro rata) + attention "
-            f"of {rows_per_head} random query rows of it ({t_rows:.2f} s) on {threads} threads")
+            f"of {what} query rows of it ({t_rows:.2f} s) on {threads} threads")
     return ops / secs / 1e12, secs, threads, text
 
 
@@ -99,10 +105,12 @@ def run_reference(args, w):
     vals = []
     x = synth.make_inputs(w)
     info = None
+    # each step: one head's quantize (charged pro rata) + 2,048 query rows, about a second
+    rows = args.cpu_sample_rows if args.cpu_sample_rows > 0 else 2048
     if args.warmup > 0:
-        cpu_oracle_sample(w, max(2, args.cpu_sample_rows // 8), x)
+        cpu_oracle_sample(w, 64, x)
     for _ in range(K):
-        tops, secs, threads, text = cpu_oracle_sample(w, max(2, args.cpu_sample_rows // 4), x)
+        tops, secs, threads, text = cpu_oracle_sample(w, rows, x)
         vals.append(tops)
         info = (threads, text)
     value = statistics.median(vals)
@@ -314,8 +322,8 @@ def run_ours(args, w):
                 "algorithmic_ops_per_launch": ops,
                 "traffic": None if tr is None else tr["dram_bytes_per_launch_full"],
                 "quantize_ms": quant_avg, "attention_ms": attn_avg,
-                "quantize_gbs": (10 * w.B * w.Tkv * w.H * w.D + 2 * w.B * w.Tq * w.H * w.D
-                                 + 3 * w.B * w.Tkv * w.H * w.D) / (quant_avg * 1e-3) / 1e9}
+                # stats reads K, V (4 B); quantize reads Q, K, V (2 + 4 B) and writes q8, k8, v8 (1 + 2 B)
+                "quantize_gbs": (10 * w.Tkv + 3 * w.Tq) * w.B * w.H * w.D / (quant_avg * 1e-3) / 1e9}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
