@@ -70,9 +70,7 @@ struct __align__(1024) AttnSmem {
   uint64_t s_full[2];   // MMA -> softmax: scores of key tile j in S(j%2)
   uint64_t s_free[2];   // softmax -> MMA: scores of key tile j read, S(j%2) may be overwritten
   uint64_t p_full[2];   // softmax -> MMA: P of key tile j in P(j%2)
-  uint64_t a_full[2];   // softmax -> correction: alpha of key tile j in alpha[j%2]
-  uint64_t a_free[2];   // correction -> softmax: alpha of key tile j read, alpha[j%2] may be rewritten
-  uint64_t m_full[2];   // softmax of tile j -> softmax of tile j+1: running max in mrow[j%2]
+  uint64_t m_full[4];   // softmax of tile j -> softmax of tile j+1 and correction: running max in mrow[j%4]
   uint64_t o_ready[2];  // correction -> MMA: O rescaled for key tile j
   uint64_t pv_done[2];  // MMA -> correction, softmax: PV of key tile j completed (P(j%2) free)
   uint64_t o_full;      // MMA -> epilogue: the last PV completed
@@ -81,8 +79,7 @@ struct __align__(1024) AttnSmem {
   uint32_t tmem_base;
   int abort;
   float sv[kD];
-  float alpha[2][kTile];
-  float mrow[2][kTile];   // [key tile parity][row]: running max after that tile (log2 domain)
+  float mrow[4][kTile];   // [key tile % 4][row]: running max after that tile (log2 domain)
   float dsum[2][kTile];   // [warpgroup][row]: sum of 448*p over its tiles, relative to mlast
   float mlast[2][kTile];  // [warpgroup][row]: running max at its last tile
 };
@@ -90,7 +87,7 @@ struct __align__(1024) AttnSmem {
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
-  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteSoftA, kSiteCorrA, kSiteCorrPV, kSiteEpi
+  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
@@ -109,11 +106,16 @@ __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int quarter, u
 constexpr uint32_t kMagic = 0x4B400000u;  // bit pattern of 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;     // 1.5 * 2^23
 constexpr float kLog2_448 = 8.80735492205760410749f;
+// Key pairs, out of every 8, whose exp2 runs on the FMA pipe instead of MUFU.
+#ifndef H3ATTN_FMA_EXP2_PAIRS_OF_8
+#define H3ATTN_FMA_EXP2_PAIRS_OF_8 2
+#endif
+constexpr int kFmaExp2PairsOf8 = H3ATTN_FMA_EXP2_PAIRS_OF_8;
 
 // The 128 INT32 scores of a row become x = 1.5*2^23 + acc as FP32 bit patterns
 // (exact, |acc| < 2^22), in place; x is monotone in acc, so the row maxima of
-// the two 64-key halves (one K scale each) are taken on x.  With kMasked,
-// columns >= valid (keys past Tkv) become 0, below every x.
+// the two 64-key halves (one K scale each) are taken on x with 3-input max.
+// With kMasked, columns >= valid (keys past Tkv) become 0, below every x.
 template <bool kMasked>
 __device__ __forceinline__ void magic_and_max(uint32_t (&s)[128], int valid, float& xm0, float& xm1) {
 #pragma unroll
@@ -160,11 +162,17 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
   q1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
 }
 
+__device__ __forceinline__ float exp2_fma(float u) {
+  float q0, q1;
+  exp2_fma_pair(f2_pack(u, u), q0, q1);
+  return q0;
+}
+
 // Scaled probabilities of the 128 keys of a row: q = 2^((x - 1.5*2^23)*f - mq)
 // with mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
-// into acc2 and the E4M3 words of q into w (4 keys per word).  One key pair in
-// four takes its exp2 from the FMA pipe (exp2_fma_pair), the rest from MUFU,
-// which balances the two units.
+// into acc2 and the E4M3 words of q into w (4 keys per word).  kFmaExp2PairsOf8
+// key pairs in every eight take their exp2 from the FMA pipe (exp2_fma_pair),
+// the rest from MUFU, to balance the two units.
 template <bool kMasked>
 __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
                                          uint64_t (&acc2)[4], uint32_t (&w)[32]) {
@@ -180,7 +188,7 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
       const uint64_t a = f2_add(f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1])), negC);
       const uint64_t u = f2_fma(a, i < 64 ? ff0 : ff1, negm);
       float q0, q1;
-      if (((i >> 1) & 3) == 3) {
+      if (((i >> 1) & 7) < kFmaExp2PairsOf8) {
         exp2_fma_pair(u, q0, q1);
       } else {
         float u0, u1;
@@ -222,7 +230,11 @@ enum : int {
   kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed (before the P store)
   kEvPVDone = 8,   // MMA issuer: PV of key tile j issued and committed
   kEvSFree = 9,    // MMA issuer: scores of key tile j released by the softmax (QK(j+2) may start)
-  kNumEvents = 10
+  kEvLd = 10,      // softmax warp: scores in registers
+  kEvMax = 11,     // softmax warp: own row maxima known (before the running-max hand-off)
+  kEvMWait = 12,   // softmax warp: running max of tile j-1 received
+  kEvAFree = 13,   // softmax warp: alpha slot released by the correction warpgroup
+  kNumEvents = 14
 };
 
 struct AttnParams {
@@ -272,9 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_free[i], kTile);
       mbar_init(&sm.pv_done[i], 1);
       mbar_init(&sm.p_full[i], kTile);
-      mbar_init(&sm.a_full[i], kTile);
-      mbar_init(&sm.a_free[i], kTile);
       mbar_init(&sm.m_full[i], kTile);
+      mbar_init(&sm.m_full[i + 2], kTile);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&sm.o_ready[i], kTile);
     mbar_init(&sm.o_full, 1);
@@ -438,15 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dealloc<kRegsCorrection>();
     const uint32_t tO = tmem_lane_addr(tmem, quarter, kColO);
     bool ok = true;
+    float m_prev = -INFINITY;  // running max after key tile j-1
     for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(&sm.a_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
+      ok = mbar_wait(&sm.m_full[j & 3], (uint32_t)(j >> 2) & 1u, abort, kWaitLimitNs);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
-        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrA, abort);
+        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrM, abort);
         break;
       }
-      const float alpha = sm.alpha[j & 1][row];
-      mbar_arrive(&sm.a_free[j & 1]);
+      const float m_j = sm.mrow[j & 3][row];
+      const float alpha = ex2_approx(__fsub_rn(m_prev, m_j));
+      m_prev = m_j;
       if (j > 0) {
         // O holds the sum over key tiles < j once the PV of tile j-1 has completed.  The
         // wait also keeps this warpgroup from running two tiles ahead of the PV issuer.
@@ -555,38 +568,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld64x2(tS, x);
       tc_fence_before();
       mbar_arrive(&sm.s_free[par]);
+      if (tr) trace(kEvLd, par, j);
       float xm0, xm1;
       if (valid < kTile)
         magic_and_max<true>(x, valid, xm0, xm1);
       else
         magic_and_max<false>(x, valid, xm0, xm1);
-      const float t0m = valid > 0 ? __fmul_rn(__fsub_rn(xm0, kMagicF), f0) : -INFINITY;
+      const float t0m = __fmul_rn(__fsub_rn(xm0, kMagicF), f0);  // valid >= 1: half 0 has a key
       const float t1m = valid > 64 ? __fmul_rn(__fsub_rn(xm1, kMagicF), f1) : -INFINITY;
+      if (tr) {
+        asm volatile("" ::"f"(t0m), "f"(t1m));  // the maxima exist before the stamp is taken
+        trace(kEvMax, par, j);
+      }
       // running max after tile j-1, from the other warpgroup
       float m_prev = -INFINITY;
       if (j > 0) {
-        ok = mbar_wait(&sm.m_full[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort, kWaitLimitNs);
+        ok = mbar_wait(&sm.m_full[(j - 1) & 3], (uint32_t)((j - 1) >> 2) & 1u, abort, kWaitLimitNs);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftM, abort);
           break;
         }
-        m_prev = sm.mrow[(j - 1) & 1][row];
+        m_prev = sm.mrow[(j - 1) & 3][row];
       }
+      if (tr) trace(kEvMWait, par, j);
       const float m_j = fmaxf(m_prev, fmaxf(t0m, t1m));
-      sm.mrow[j & 1][row] = m_j;
-      mbar_arrive(&sm.m_full[j & 1]);
-      if (j >= 2) {
-        // the correction warpgroup has read alpha of tile j-2 from this slot
-        ok = mbar_wait(&sm.a_free[par], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) {
-          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftA, abort);
-          break;
-        }
-      }
-      sm.alpha[j & 1][row] = ex2_approx(__fsub_rn(m_prev, m_j));
-      mbar_arrive(&sm.a_full[j & 1]);
+      sm.mrow[j & 3][row] = m_j;
+      mbar_arrive(&sm.m_full[j & 3]);
       if (tr) trace(kEvAlpha, par, j);
       uint32_t pw[32];
       uint64_t acc2[4];
@@ -617,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
       const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-      d_w = __fadd_rn(__fmul_rn(d_w, ex2_approx(__fsub_rn(m_w, m_j))), es);
+      d_w = __fadd_rn(__fmul_rn(d_w, exp2_fma(__fsub_rn(m_w, m_j))), es);
       m_w = m_j;
     }
     if (ok) {
