@@ -80,8 +80,10 @@ typedef struct {
 /* Workspace fields, in the order h3attn_workspace_layout reports their byte offsets. */
 enum {
   H3ATTN_WS_STATUS = 0, /* int32 status word (+ detail words), 256 bytes */
-  H3ATTN_WS_Q8,         /* int8  [B, H, Tq_pad, 128]   Tq_pad  = ceil(Tq/128)*128, rows >= Tq are 0 */
-  H3ATTN_WS_K8,         /* int8  [B, H, Tkv_pad, 128]  Tkv_pad = ceil(Tkv/128)*128, rows >= Tkv are 0 */
+  H3ATTN_WS_Q8,         /* INT8 Q words held as BF16 values (exact), [B, H, Tq_pad, 128];
+                           Tq_pad = ceil(Tq/128)*128, rows >= Tq are 0 */
+  H3ATTN_WS_K8,         /* INT8 K words held as BF16 values, [B, H, Tkv_pad, 128];
+                           Tkv_pad = ceil(Tkv/128)*128, rows >= Tkv are 0 */
   H3ATTN_WS_V8T,        /* e4m3  [B, H, 128, Tkv_pad]  V transposed (channel-major), columns >= Tkv are 0 */
   H3ATTN_WS_SQ,         /* f32   [B, H, Tq_pad/32]     Q group scales (0 for groups past Tq) */
   H3ATTN_WS_SK,         /* f32   [B, H, Tkv_pad/64]    K group scales (0 for groups past Tkv) */
@@ -110,9 +112,11 @@ h3attn_status h3attn_quantize_qkv(const h3attn_bf16_view* q, const h3attn_bf16_v
                                   void* ws, size_t ws_bytes, void* stream);
 
 /* The fused attention mainloop on a workspace filled by h3attn_quantize_qkv with the
- * same sizes: INT8 QK^T on the tensor cores into tensor memory, FP32 online softmax,
- * FP8 P, FP8 PV with FP32 accumulation, final reciprocal, BF16 store of rows < Tq
- * into `out`.  softmax_scale is usually 1/sqrt(D). */
+ * same sizes: QK^T of the INT8 words on the tensor cores into tensor memory (BF16
+ * operands holding the integers, FP32 accumulation: exact, since every product and
+ * partial sum is an integer below 2^24), FP32 online softmax, FP8 P, FP8 PV with FP32
+ * accumulation, final reciprocal, BF16 store of rows < Tq into `out`.
+ * softmax_scale is usually 1/sqrt(D). */
 h3attn_status h3attn_attend(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H, int D,
                             float softmax_scale, const h3attn_bf16_out* out, void* stream);
 

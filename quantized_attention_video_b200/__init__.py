@@ -210,7 +210,7 @@ def h3attn_debug_attend_trace(ws, B: int, Tq: int, Tkv: int, H: int, softmax_sca
 
 
 def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:
-    """Typed views of the workspace fields (for parity checks)."""
+    """Typed views of the workspace fields (for parity checks; q8/k8 are INT8 copies)."""
     import torch
     off = h3attn_workspace_layout(B, Tq, Tkv, H)
     Tqp, Tkp = -(-Tq // TILE) * TILE, -(-Tkv // TILE) * TILE
@@ -220,9 +220,10 @@ def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:
         return ws[off[name]:off[name] + nb].view(dtype).view(shape)
 
     BH = B * H
+    # the INT8 Q/K words are stored as BF16 values (exact); inspect them as INT8
     return dict(
-        q8=sl("q8", BH * Tqp * 128, torch.int8, (B, H, Tqp, 128)),
-        k8=sl("k8", BH * Tkp * 128, torch.int8, (B, H, Tkp, 128)),
+        q8=sl("q8", BH * Tqp * 128, torch.bfloat16, (B, H, Tqp, 128)).to(torch.int8),
+        k8=sl("k8", BH * Tkp * 128, torch.bfloat16, (B, H, Tkp, 128)).to(torch.int8),
         v8t=sl("v8t", BH * 128 * Tkp, torch.uint8, (B, H, 128, Tkp)),
         sq=sl("sq", BH * (Tqp // Q_GROUP), torch.float32, (B, H, Tqp // Q_GROUP)),
         sk=sl("sk", BH * (Tkp // K_GROUP), torch.float32, (B, H, Tkp // K_GROUP)),

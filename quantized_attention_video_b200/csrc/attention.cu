@@ -4,11 +4,13 @@
 //
 // One CTA owns one 128-row Q tile of one (b, h) and streams all 128-key K/V
 // tiles past it.  Warp roles (512 threads, four warpgroups):
-//   WG0  warp 0   TMA producer of the Q tile and the K tiles (4-stage ring).
+//   WG0  warp 0   TMA producer of the Q tile and the K tiles (3-stage ring).
 //        warp 2   TMA producer of the V^T tiles (4-stage ring), so K tiles
 //                 run ahead of V tiles by as much as the rings allow.
 //        warp 1   tensor-memory allocator and QK issuer (one thread):
-//                 S = Q K^T  tcgen05.mma kind::i8 (INT8 x INT8 -> S32).
+//                 S = Q K^T  tcgen05.mma kind::f16 on the INT8 words held as
+//                 BF16 (exact) with FP32 accumulation: every product and partial
+//                 sum is an integer below 2^24, so S equals the INT32 scores.
 //        warp 3   PV issuer (one thread):
 //                 O += P V   tcgen05.mma kind::f8f6f4 (E4M3, A = P read from
 //                 tensor memory, F32 accumulate).
@@ -23,7 +25,7 @@
 //   WG3  O correction (rescale by alpha when the running max moves) and the
 //        epilogue (final reciprocal, BF16 store).
 // Tensor memory (512 columns allocated): S0 [0,128) S1 [128,256) O [256,384)
-// P0 [384,416) P1 [416,448).  Scores of key tile j go to S(j%2) and its E4M3
+// P0 [384,416) P1 [416,448).  FP32 scores of key tile j go to S(j%2) and its E4M3
 // probabilities (128 x 128 bytes = 32 columns) to P(j%2).  The softmax frees
 // S(j%2) as soon as it has read the scores, so QK(j+2) runs on the tensor
 // cores while the softmax of tile j is still computing; it writes P(j%2)
@@ -47,11 +49,13 @@
 namespace h3 {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStagesK = 3;  // K ring (BF16 tiles, 32 KB each)
+constexpr int kStagesV = 4;  // V ring (E4M3 tiles, 16 KB each)
 constexpr int kThreads = 512;
-constexpr uint32_t kTileBytes = 128 * 128;
+constexpr uint32_t kTileBytes = 128 * 128;          // one 128 x 128-byte swizzled tile
+constexpr uint32_t kQKTileBytes = 2 * kTileBytes;   // a BF16 128 x 128 tile: two 64-column halves
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 416;
-constexpr uint32_t kIdescQK = idesc_i8_s32(128, 128);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // setmaxnreg split (registers per thread): control, correction, softmax warpgroups.
@@ -61,12 +65,12 @@ static_assert(kRegSplitTotal <= 65536, "register split exceeds the SM register f
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 
 struct __align__(1024) AttnSmem {
-  uint8_t q[kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t q[2][kTileBytes];            // BF16 Q tile: key dims [0,64) and [64,128)
+  uint8_t k[kStagesK][2][kTileBytes];  // BF16 K tiles, same split
+  uint8_t v[kStagesV][kTileBytes];     // E4M3 V^T tiles
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kStagesK], k_empty[kStagesK];
+  uint64_t v_full[kStagesV], v_empty[kStagesV];
   uint64_t s_full[2];   // MMA -> softmax: scores of key tile j in S(j%2)
   uint64_t s_free[2];   // softmax -> MMA: scores of key tile j read, S(j%2) may be overwritten
   uint64_t p_full[2];   // softmax -> MMA: P of key tile j in P(j%2)
@@ -103,8 +107,7 @@ __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int quarter, u
   return base + ((uint32_t)(32 * quarter) << 16) + col;
 }
 
-constexpr uint32_t kMagic = 0x4B400000u;  // bit pattern of 1.5 * 2^23
-constexpr float kMagicF = 12582912.0f;     // 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23: float + magic rounds to an integer
 constexpr float kLog2_448 = 8.80735492205760410749f;
 // Key pairs, out of every 8, whose exp2 runs on the FMA pipe instead of MUFU.
 #ifndef H3ATTN_FMA_EXP2_PAIRS_OF_8
@@ -112,25 +115,23 @@ constexpr float kLog2_448 = 8.80735492205760410749f;
 #endif
 constexpr int kFmaExp2PairsOf8 = H3ATTN_FMA_EXP2_PAIRS_OF_8;
 
-// The 128 INT32 scores of a row become x = 1.5*2^23 + acc as FP32 bit patterns
-// (exact, |acc| < 2^22), in place; x is monotone in acc, so the row maxima of
-// the two 64-key halves (one K scale each) are taken on x with 3-input max.
-// With kMasked, columns >= valid (keys past Tkv) become 0, below every x.
+// Row maxima of the two 64-key halves (one K scale each) of the 128 FP32
+// scores of a row (integer-valued: the exact INT32 dot products), with 3-input
+// max; with kMasked, columns >= valid (keys past Tkv) are ignored.
 template <bool kMasked>
-__device__ __forceinline__ void magic_and_max(uint32_t (&s)[128], int valid, float& xm0, float& xm1) {
-#pragma unroll
-  for (int e = 0; e < 128; ++e) {
-    uint32_t v = s[e] + kMagic;
-    if (kMasked && e >= valid) v = 0u;
-    s[e] = v;
-  }
+__device__ __forceinline__ void rowmax128(const uint32_t (&s)[128], int valid, float& xm0, float& xm1) {
   float m[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) m[c] = 0.0f;
+  for (int c = 0; c < 8; ++c) m[c] = -INFINITY;
 #pragma unroll
   for (int e = 0; e < 128; e += 2) {
     const int c = ((e >> 1) & 3) + (e >= 64 ? 4 : 0);
-    m[c] = fmax3(m[c], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+    float a = __uint_as_float(s[e]), b = __uint_as_float(s[e + 1]);
+    if (kMasked) {
+      if (e >= valid) a = -INFINITY;
+      if (e + 1 >= valid) b = -INFINITY;
+    }
+    m[c] = fmax3(m[c], a, b);
   }
   xm0 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
   xm1 = fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7]));
@@ -168,15 +169,14 @@ __device__ __forceinline__ float exp2_fma(float u) {
   return q0;
 }
 
-// Scaled probabilities of the 128 keys of a row: q = 2^((x - 1.5*2^23)*f - mq)
-// with mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
+// Scaled probabilities of the 128 keys of a row: q = 2^(acc*f - mq) with
+// mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
 // into acc2 and the E4M3 words of q into w (4 keys per word).  kFmaExp2PairsOf8
 // key pairs in every eight take their exp2 from the FMA pipe (exp2_fma_pair),
 // the rest from MUFU, to balance the two units.
 template <bool kMasked>
 __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
                                          uint64_t (&acc2)[4], uint32_t (&w)[32]) {
-  const uint64_t negC = f2_pack(-kMagicF, -kMagicF);
   const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
   const uint64_t negm = f2_pack(-mq, -mq);
 #pragma unroll
@@ -185,7 +185,7 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int i = e + 2 * hp;
-      const uint64_t a = f2_add(f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1])), negC);
+      const uint64_t a = f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1]));
       const uint64_t u = f2_fma(a, i < 64 ? ff0 : ff1, negm);
       float q0, q1;
       if (((i >> 1) & 7) < kFmaExp2PairsOf8) {
@@ -273,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ set-up ----
   if (warp == 0 && lane == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
@@ -318,25 +320,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-        tma_load_2d(sm.q, &tm_q, &sm.q_full, 0, (int)(bh * p.Tq_pad + (int64_t)qt * kTile));
+        const int qrow = (int)(bh * p.Tq_pad + (int64_t)qt * kTile);
+        mbar_arrive_expect_tx(&sm.q_full, kQKTileBytes);
+        tma_load_2d(sm.q[0], &tm_q, &sm.q_full, 0, qrow);
+        tma_load_2d(sm.q[1], &tm_q, &sm.q_full, 64, qrow);
         const int krow = (int)(bh * p.Tkv_pad);
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
-          const int s = j % kStages;
-          if (!mbar_wait(&sm.k_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort, kWaitLimitNs)) {
+          const int s = j % kStagesK;
+          if (!mbar_wait(&sm.k_empty[s], ((uint32_t)(j / kStagesK) & 1u) ^ 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdKEmpty, abort);
             break;
           }
-          mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
-          tma_load_2d(sm.k[s], &tm_k, &sm.k_full[s], 0, krow + j * kTile);
+          mbar_arrive_expect_tx(&sm.k_full[s], kQKTileBytes);
+          tma_load_2d(sm.k[s][0], &tm_k, &sm.k_full[s], 0, krow + j * kTile);
+          tma_load_2d(sm.k[s][1], &tm_k, &sm.k_full[s], 64, krow + j * kTile);
           issued = j + 1;
         }
         if (*abort) {
           // let every copy this thread started land before the CTA can exit
           mbar_wait(&sm.q_full, 0, nullptr, kDrainLimitNs);
-          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-            mbar_wait(&sm.k_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, kDrainLimitNs);
+          for (int j = (issued > kStagesK ? issued - kStagesK : 0); j < issued; ++j)
+            mbar_wait(&sm.k_full[j % kStagesK], (uint32_t)(j / kStagesK) & 1u, nullptr, kDrainLimitNs);
         }
       }
       __syncwarp();
@@ -347,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int vrow = (int)(bh * kD);
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
-          const int s = j % kStages;
-          if (!mbar_wait(&sm.v_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort, kWaitLimitNs)) {
+          const int s = j % kStagesV;
+          if (!mbar_wait(&sm.v_empty[s], ((uint32_t)(j / kStagesV) & 1u) ^ 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdVEmpty, abort);
             break;
           }
@@ -357,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued = j + 1;
         }
         if (*abort) {
-          for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-            mbar_wait(&sm.v_full[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, kDrainLimitNs);
+          for (int j = (issued > kStagesV ? issued - kStagesV : 0); j < issued; ++j)
+            mbar_wait(&sm.v_full[j % kStagesV], (uint32_t)(j / kStagesV) & 1u, nullptr, kDrainLimitNs);
         }
       }
       __syncwarp();
@@ -368,9 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = mbar_wait(&sm.q_full, 0, abort, kWaitLimitNs);
         if (!ok) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaQ, abort);
         tc_fence_after();
-        const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q));
         for (int j = 0; ok && j < nkv; ++j) {
-          const int s = j % kStages;
+          const int s = j % kStagesK;
           if (j >= 2) {
             // S(j%2) is free once the softmax of tile j-2 has read its scores
             if (!mbar_wait(&sm.s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs)) {
@@ -381,17 +385,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             trace(kEvSFree, 0, j - 2);
           }
-          if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStages) & 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStagesK) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
             ok = false;
             break;
           }
           tc_fence_after();
           trace(kEvKFull, 0, j);
-          const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s]));
           const uint32_t s_col = (j & 1) ? kColS1 : kColS0;
+          // 8 MMAs of K = 16: BF16 key dims [16kk, 16kk+16) = bytes 32*(kk%4) of half kk/4
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem + s_col, dq + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q[kk >> 2])) + 2 * (kk & 3);
+            const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s][kk >> 2])) + 2 * (kk & 3);
+            mma_bf16_ss(tmem + s_col, dq, dk, kIdescQK, kk > 0);
+          }
           mma_commit(&sm.s_full[j & 1]);
           mma_commit(&sm.k_empty[s]);
           trace(kEvQK, 0, j);
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
-          const int s = j % kStages;
+          const int s = j % kStagesV;
           if (!mbar_wait(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
             ok = false;
@@ -417,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStages) & 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStagesV) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaV, abort);
             ok = false;
             break;
@@ -571,11 +579,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tr) trace(kEvLd, par, j);
       float xm0, xm1;
       if (valid < kTile)
-        magic_and_max<true>(x, valid, xm0, xm1);
+        rowmax128<true>(x, valid, xm0, xm1);
       else
-        magic_and_max<false>(x, valid, xm0, xm1);
-      const float t0m = __fmul_rn(__fsub_rn(xm0, kMagicF), f0);  // valid >= 1: half 0 has a key
-      const float t1m = valid > 64 ? __fmul_rn(__fsub_rn(xm1, kMagicF), f1) : -INFINITY;
+        rowmax128<false>(x, valid, xm0, xm1);
+      const float t0m = __fmul_rn(xm0, f0);  // valid >= 1: half 0 has a key
+      const float t1m = valid > 64 ? __fmul_rn(xm1, f1) : -INFINITY;
       if (tr) {
         asm volatile("" ::"f"(t0m), "f"(t1m));  // the maxima exist before the stamp is taken
         trace(kEvMax, par, j);
@@ -638,11 +646,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------- debug QK tile ----
-// One CTA of 128 threads computes the INT32 QK^T tile of (b, h, qt, kt) with
-// the same TMA + tcgen05 kind::i8 path and writes it to global memory.
+// One CTA of 128 threads computes the QK^T tile of (b, h, qt, kt) with the
+// same TMA + tcgen05 path as the attention kernel and writes it to global
+// memory as INT32 (the FP32 scores are exact integers).
 struct __align__(1024) DebugSmem {
-  uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
+  uint8_t q[2][kTileBytes];
+  uint8_t k[2][kTileBytes];
   uint64_t full, done;
   uint32_t tmem_base;
   int abort;
@@ -670,14 +679,19 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&sm.full, 2 * kTileBytes);
-    tma_load_2d(sm.q, &tm_q, &sm.full, 0, qrow);
-    tma_load_2d(sm.k, &tm_k, &sm.full, 0, krow);
+    mbar_arrive_expect_tx(&sm.full, 2 * kQKTileBytes);
+    tma_load_2d(sm.q[0], &tm_q, &sm.full, 0, qrow);
+    tma_load_2d(sm.q[1], &tm_q, &sm.full, 64, qrow);
+    tma_load_2d(sm.k[0], &tm_k, &sm.full, 0, krow);
+    tma_load_2d(sm.k[1], &tm_k, &sm.full, 64, krow);
     if (mbar_wait(&sm.full, 0, nullptr, kWaitLimitNs)) {
       tc_fence_after();
-      const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q)), dk = sdesc_k_sw128(smem_u32(sm.k));
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) mma_i8_ss(tmem, dq + 2 * kk, dk + 2 * kk, kIdescQK, kk > 0);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q[kk >> 2])) + 2 * (kk & 3);
+        const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[kk >> 2])) + 2 * (kk & 3);
+        mma_bf16_ss(tmem, dq, dk, kIdescQK, kk > 0);
+      }
       mma_commit(&sm.done);
     } else {
       record_failure(status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
@@ -693,7 +707,8 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t a[32];
       tmem_ld32(tmem_lane_addr(tmem, warp, 32 * ch), a);
       tmem_wait_ld();
-      for (int e = 0; e < 32; ++e) out[row * 128 + 32 * ch + e] = (int32_t)a[e];
+      // the FP32 scores are integers below 2^24: exact INT32 values
+      for (int e = 0; e < 32; ++e) out[row * 128 + 32 * ch + e] = __float2int_rn(__uint_as_float(a[e]));
     }
   } else if (lane == 0) {
     record_failure(status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
@@ -724,15 +739,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D byte tensor [rows, inner] with a row pitch; 128 x 128-byte boxes, 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch) {
+// 2D tensor [rows, inner] (inner in elements) with a row pitch in bytes; boxes of
+// 128 rows x 128 bytes, 128-byte swizzle.  8-bit data (UINT8) or BF16.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch, bool bf16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {pitch};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {bf16 ? 64u : 128u, 128};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+            dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -775,8 +792,8 @@ cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, fl
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv;
   const uint64_t BH = (uint64_t)s.B * s.H;
-  if (!make_tmap(&tq, ws + L.off[H3ATTN_WS_Q8], kD, BH * s.Tq_pad, kD) ||
-      !make_tmap(&tk, ws + L.off[H3ATTN_WS_K8], kD, BH * s.Tkv_pad, kD) ||
+  if (!make_tmap(&tq, ws + L.off[H3ATTN_WS_Q8], kD, BH * s.Tq_pad, 2 * kD, true) ||
+      !make_tmap(&tk, ws + L.off[H3ATTN_WS_K8], kD, BH * s.Tkv_pad, 2 * kD, true) ||
       !make_tmap(&tv, ws + L.off[H3ATTN_WS_V8T], s.Tkv_pad, BH * kD, s.Tkv_pad)) {
     *why = H3ATTN_ERR_CUDA;
     return cudaErrorInvalidValue;
@@ -813,8 +830,8 @@ cudaError_t launch_debug_qk(const char* ws, const Shape& s, const Layout& L, int
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk;
   const uint64_t BH = (uint64_t)s.B * s.H;
-  if (!make_tmap(&tq, ws + L.off[H3ATTN_WS_Q8], kD, BH * s.Tq_pad, kD) ||
-      !make_tmap(&tk, ws + L.off[H3ATTN_WS_K8], kD, BH * s.Tkv_pad, kD)) {
+  if (!make_tmap(&tq, ws + L.off[H3ATTN_WS_Q8], kD, BH * s.Tq_pad, 2 * kD, true) ||
+      !make_tmap(&tk, ws + L.off[H3ATTN_WS_K8], kD, BH * s.Tkv_pad, 2 * kD, true)) {
     *why = H3ATTN_ERR_CUDA;
     return cudaErrorInvalidValue;
   }

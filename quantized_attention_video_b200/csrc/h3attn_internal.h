@@ -39,8 +39,8 @@ inline Layout make_layout(const Shape& s) {
   const int64_t BH = (int64_t)s.B * s.H;
   int64_t sz[H3ATTN_WS_NFIELDS] = {};
   sz[H3ATTN_WS_STATUS] = 256;
-  sz[H3ATTN_WS_Q8] = BH * s.Tq_pad * kD;
-  sz[H3ATTN_WS_K8] = BH * s.Tkv_pad * kD;
+  sz[H3ATTN_WS_Q8] = BH * s.Tq_pad * kD * 2;   // INT8 words held as equal BF16 values
+  sz[H3ATTN_WS_K8] = BH * s.Tkv_pad * kD * 2;
   sz[H3ATTN_WS_V8T] = BH * kD * s.Tkv_pad;
   sz[H3ATTN_WS_SQ] = BH * (s.Tq_pad / kQGroup) * 4;
   sz[H3ATTN_WS_SK] = BH * (s.Tkv_pad / kKGroup) * 4;

@@ -9,7 +9,11 @@
 //   quantize_kernel : one pass over Q, K, V in 128-token slabs. INT8 Q per
 //                     32-token group, INT8 (K - mean) per 64-token group, FP8 E4M3
 //                     V per channel written transposed (channel-major), zero
-//                     padding up to the 128-token tile multiple.
+//                     padding up to the 128-token tile multiple.  The INT8 Q/K
+//                     words are stored as BF16 values (every integer in [-127, 127]
+//                     is exact in BF16) so that the attention kernel can take QK^T
+//                     on the BF16 tensor-core path with FP32 scores that equal the
+//                     INT32 dot products exactly.
 //
 // All loads are 16-byte vectors of 8 BF16 channels; 16 threads cover one
 // 128-channel row, so a warp reads two contiguous 256-byte rows per load.
@@ -100,10 +104,21 @@ __global__ void __launch_bounds__(128) finalize_kernel(const double* __restrict_
 }
 
 // --------------------------------------------------------------- quantize ----
-__device__ __forceinline__ int8_t q_i8(float x, float inv) {
+__device__ __forceinline__ int q_i8(float x, float inv) {
   int r = __float2int_rn(__fmul_rn(x, inv));
-  r = max(-127, min(127, r));
-  return (int8_t)r;
+  return max(-127, min(127, r));
+}
+
+// BF16 bit pattern of a small integer (|v| <= 127: exact).
+__device__ __forceinline__ uint32_t bf16_of_int(int v) { return __float_as_uint(__int2float_rn(v)) >> 16; }
+
+// Eight quantized values of one row slice as BF16 words, one 16-byte store.
+__device__ __forceinline__ void store_words(uint16_t* dst, const float (&x)[8], float inv) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    w[e] = bf16_of_int(q_i8(x[2 * e], inv)) | (bf16_of_int(q_i8(x[2 * e + 1], inv)) << 16);
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 __device__ __forceinline__ float warp_max(float x) {
@@ -120,7 +135,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     const uint16_t* __restrict__ v, int64_t vsb, int64_t vst, int64_t vsh,
     int H, int Tq, int Tkv, int64_t Tq_pad, int64_t Tkv_pad, int64_t nchunk,
     const float* __restrict__ km, const float* __restrict__ vmax,
-    int8_t* __restrict__ q8, float* __restrict__ sq, int8_t* __restrict__ k8, float* __restrict__ sk,
+    uint16_t* __restrict__ q8, float* __restrict__ sq, uint16_t* __restrict__ k8, float* __restrict__ sk,
     uint8_t* __restrict__ v8t) {
   __shared__ float red[8];
   __shared__ float gmax[4];
@@ -162,13 +177,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int64_t t = t0 + 8 * rq + r;
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w0 |= (uint32_t)(uint8_t)q_i8(x[r][e], inv) << (8 * e);
-        w1 |= (uint32_t)(uint8_t)q_i8(x[r][e + 4], inv) << (8 * e);
-      }
-      *reinterpret_cast<uint2*>(q8 + (bh * Tq_pad + t) * kD + c16 * 8) = make_uint2(w0, w1);
+      store_words(q8 + (bh * Tq_pad + t) * kD + c16 * 8, x[r], inv);
     }
     __syncthreads();
   }
@@ -209,13 +218,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int64_t t = t0 + 8 * rq + r;
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w0 |= (uint32_t)(uint8_t)q_i8(x[r][e], inv) << (8 * e);
-        w1 |= (uint32_t)(uint8_t)q_i8(x[r][e + 4], inv) << (8 * e);
-      }
-      *reinterpret_cast<uint2*>(k8 + (bh * Tkv_pad + t) * kD + c16 * 8) = make_uint2(w0, w1);
+      store_words(k8 + (bh * Tkv_pad + t) * kD + c16 * 8, x[r], inv);
     }
   }
   // ---------------------------------------------------------------- V ----
@@ -292,8 +295,8 @@ cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k
       static_cast<const uint16_t*>(q.data), q.stride_b, q.stride_t, q.stride_h,
       static_cast<const uint16_t*>(k.data), k.stride_b, k.stride_t, k.stride_h,
       static_cast<const uint16_t*>(v.data), v.stride_b, v.stride_t, v.stride_h, s.H, s.Tq, s.Tkv, s.Tq_pad,
-      s.Tkv_pad, s.nchunk, km, vmax, reinterpret_cast<int8_t*>(ws + L.off[H3ATTN_WS_Q8]),
-      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SQ]), reinterpret_cast<int8_t*>(ws + L.off[H3ATTN_WS_K8]),
+      s.Tkv_pad, s.nchunk, km, vmax, reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_Q8]),
+      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SQ]), reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_K8]),
       reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SK]), reinterpret_cast<uint8_t*>(ws + L.off[H3ATTN_WS_V8T]));
   return cudaGetLastError();
 }

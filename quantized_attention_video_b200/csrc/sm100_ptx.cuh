@@ -129,6 +129,16 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] x B[smem desc]^T, BF16 operands, F32 accumulate.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] x B[smem desc]^T, FP8 E4M3 operands, F32 accumulate.
 __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -363,10 +373,13 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
 }
 
 // Instruction descriptor: D format in bits 4-5 (1 = F32, 2 = S32), A format in
-// 7-9, B format in 10-12 (8-bit integer: 1 = signed; FP8: 0 = E4M3), both
+// 7-9, B format in 10-12 (8-bit integer: 1 = signed; FP8: 0 = E4M3; 16-bit: 1 = BF16), both
 // operands K-major (bits 15, 16 = 0), N >> 3 in 17-22, M >> 4 in 24-28.
 __host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);

@@ -46,7 +46,8 @@ def test_workspace_layout_matches_field_sizes(L):
     off = h3.h3attn_workspace_layout(B, Tq, Tkv, H)
     Tqp, Tkp = 384, 9472
     nchunk = -(-Tkv // 64)
-    need = {"status": 256, "q8": B * H * Tqp * 128, "k8": B * H * Tkp * 128, "v8t": B * H * 128 * Tkp,
+    # the INT8 Q/K words are held as BF16 values (2 bytes each)
+    need = {"status": 256, "q8": 2 * B * H * Tqp * 128, "k8": 2 * B * H * Tkp * 128, "v8t": B * H * 128 * Tkp,
             "sq": B * H * Tqp // 32 * 4, "sk": B * H * Tkp // 64 * 4, "km": B * H * 128 * 4,
             "sv": B * H * 128 * 4, "ksum": B * H * nchunk * 128 * 8, "vmax": B * H * nchunk * 128 * 4}
     names = h3.WS_FIELDS
