@@ -145,15 +145,17 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
 
 /* Tracing export: h3attn_attend with a timeline probe in one CTA (linear block index
  * trace_block; CTAs are (Q tile, head, batch), Q tile fastest).  Writes clock64()
- * stamps of 14 events for each key tile j to trace_dev[(event*2 + slot)*ceil(Tkv/128) + j]
- * (uint64, device memory, 28*ceil(Tkv/128) entries; entries of events that did not
+ * stamps of 16 events for each key tile j to trace_dev[(event*2 + slot)*ceil(Tkv/128) + j]
+ * (uint64, device memory, 32*ceil(Tkv/128) entries; entries of events that did not
  * happen are left untouched).  Softmax events use slot = j % 2 (the warpgroup that owns
  * tile j), the others slot 0.  Events: 0 scores ready in the softmax warp, 1 running max
- * and alpha published, 2 probabilities handed to the MMA issuer, 3 QK issued, 4 PV
- * issued, 5 O rescaled by the correction warp, 6 K tile landed, 7 probabilities computed,
- * 8 PV issued and committed, 9 scores released (the next QK into that buffer may start),
- * 10 scores in registers, 11 own row maxima known, 12 running max of tile j-1 received,
- * 13 alpha slot free.  Reproduces the QK/PV overlap measurement of "Phase 2B
+ * of tile j published, 2 probabilities handed to the MMA issuer, 3 QK issued, 4 PV
+ * issued, 5 O rescaled (or left alone) by the correction warp, 6 K tile landed,
+ * 7 probabilities computed, 8 PV issued and committed, 9 scores released (the next QK
+ * into that buffer may start), 10 scores in registers, 11 own row maxima known,
+ * 12 running max of tile j-1 received, 13 the PV issuer saw the probabilities, 14 the PV
+ * issuer saw O ready, 15 probabilities handed over by the softmax warp of the last row
+ * quarter (event 2 is the first quarter's).  Reproduces the QK/PV overlap measurement of "Phase 2B
  * Aligned Numerical Prototype", Synchronization And Safety.  Same output as h3attn_attend. */
 h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H,
                                         int D, float softmax_scale, const h3attn_bf16_out* out,

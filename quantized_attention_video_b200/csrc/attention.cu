@@ -233,9 +233,12 @@ enum : int {
   kEvLd = 10,      // softmax warp: scores in registers
   kEvMax = 11,     // softmax warp: own row maxima known (before the running-max hand-off)
   kEvMWait = 12,   // softmax warp: running max of tile j-1 received
-  kEvAFree = 13,   // softmax warp: alpha slot released by the correction warpgroup
-  kNumEvents = 14
+  kEvPVP = 13,     // MMA issuer: probabilities of key tile j observed (p_full)
+  kEvPVO = 14,     // MMA issuer: O ready for key tile j observed (o_ready)
+  kEvPDoneLast = 15,  // softmax warp of the last row quarter: probabilities handed over
+  kNumEvents = 16
 };
+static_assert(kNumEvents == kTraceEvents, "trace buffer layout");
 
 struct AttnParams {
   const float* sq;   // [B,H,Tq_pad/32]
@@ -420,11 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          trace(kEvPVP, 0, j);
           if (!mbar_wait(&sm.o_ready[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
             ok = false;
             break;
           }
+          trace(kEvPVO, 0, j);
           if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStagesV) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaV, abort);
             ok = false;
@@ -469,15 +474,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = ex2_approx(__fsub_rn(m_prev, m_j));
       m_prev = m_j;
       if (j > 0) {
-        // O holds the sum over key tiles < j once the PV of tile j-1 has completed.  The
-        // wait also keeps this warpgroup from running two tiles ahead of the PV issuer.
-        ok = mbar_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort, kWaitLimitNs);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) {
-          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
-          break;
+        // A warp whose rows all kept their maximum leaves O alone: PV(j) may follow
+        // PV(j-1) in the tensor pipe directly.  It still waits for PV(j-2), which
+        // consumed the previous phase of o_ready[j%2], so that this warpgroup never
+        // runs two phases ahead of the PV issuer.  A warp that rescales needs O to
+        // hold the sum over key tiles < j, i.e. PV(j-1) completed.
+        const bool rescale = __any_sync(0xFFFFFFFFu, alpha != 1.0f);
+        const int jw = rescale ? j - 1 : j - 2;
+        if (jw >= 0) {
+          ok = mbar_wait(&sm.pv_done[jw & 1], (uint32_t)(jw >> 1) & 1u, abort, kWaitLimitNs);
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          if (!ok) {
+            if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
+            break;
+          }
         }
-        if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+        if (rescale) {
           tc_fence_after();
           const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
@@ -629,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.p_full[par]);
       if (tr) trace(kEvPDone, par, j);
+      if (kTrace && tracing && quarter == 3 && lane == 0) trace(kEvPDoneLast, par, j);
       float a[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);

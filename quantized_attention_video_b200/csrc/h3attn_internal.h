@@ -74,7 +74,7 @@ struct TmapSet;  // opaque; attention.cu
 cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
                              const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why,
                              uint64_t* trace = nullptr, int trace_block = -1);
-constexpr int kTraceEvents = 14;  // events per (tile slot, key tile) in the timeline trace
+constexpr int kTraceEvents = 16;  // events per (tile slot, key tile) in the timeline trace
 cudaError_t launch_debug_qk(const char* ws, const Shape& s, const Layout& L, int b, int h, int qt, int kt,
                             int32_t* out, cudaStream_t st, h3attn_status* why);
 
