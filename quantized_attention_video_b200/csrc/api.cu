@@ -181,7 +181,7 @@ h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, 
   if (reinterpret_cast<uintptr_t>(trace_dev) % 8 != 0) return H3ATTN_ERR_ALIGNMENT;
   const Shape s = make_shape(B, Tq, Tkv, H);
   const Layout L = make_layout(s);
-  const int64_t ctas = (s.Tq_pad / kTile) * (int64_t)H * B;
+  const int64_t ctas = attention_ctas(s);
   if (trace_block < 0 || trace_block >= ctas) return H3ATTN_ERR_INVALID_ARG;
   H3_TRY(check_ws(ws, ws_bytes, L));
   H3_TRY(check_device());

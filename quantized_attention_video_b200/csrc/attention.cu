@@ -2,40 +2,40 @@
 // Phase 4: Dense Sage-Compatible Attention; numerical checkpoints of "Phase 2B
 // Aligned Numerical Prototype", Exactness).
 //
-// One CTA owns one 128-row Q tile of one (b, h) and streams all 128-key K/V
-// tiles past it.  Warp roles (512 threads, four warpgroups):
-//   WG0  warp 0   TMA producer of the Q tile and the K tiles (3-stage ring).
-//        warp 2   TMA producer of the V^T tiles (4-stage ring), so K tiles
-//                 run ahead of V tiles by as much as the rings allow.
+// One CTA owns two 128-row Q tiles (A and B) of one (b, h) and streams all
+// 128-key K/V tiles past both, so every K/V tile crosses L2 -> shared memory
+// once per 256 query rows.  Warp roles (512 threads, four warpgroups):
+//   WG0  warp 0   TMA producer of the Q tiles and the K tiles (2-stage ring).
+//        warp 2   TMA producer of the V^T tiles (3-stage ring).
 //        warp 1   tensor-memory allocator and QK issuer (one thread):
-//                 S = Q K^T  tcgen05.mma kind::f16 on the INT8 words held as
-//                 BF16 (exact) with FP32 accumulation: every product and partial
-//                 sum is an integer below 2^24, so S equals the INT32 scores.
+//                 S(x) = Q(x) K^T  tcgen05.mma kind::f16 on the INT8 words held
+//                 as BF16 (exact) with FP32 accumulation: every product and
+//                 partial sum is an integer below 2^24, so S equals the INT32
+//                 scores.
 //        warp 3   PV issuer (one thread):
-//                 O += P V   tcgen05.mma kind::f8f6f4 (E4M3, A = P read from
-//                 tensor memory, F32 accumulate).
+//                 O(x) += P(x) V   tcgen05.mma kind::f8f6f4 (E4M3 operands from
+//                 shared memory, F32 accumulate).
 //                 A tcgen05.mma issue blocks for about its execution time, so
 //                 the two products have their own issuing threads and neither
-//                 waits behind the other's dependencies.  Their MMAs touch
-//                 disjoint tensor memory; every true dependency is a barrier.
-//   WG1  softmax of the even key tiles (scores in S0)  } thread = one Q row.
-//   WG2  softmax of the odd key tiles (scores in S1)   } The running row max
-//        is handed from the warpgroup of tile j to that of tile j+1, so one
-//        warpgroup's max/exchange phase overlaps the other's exp2 phase.
-//   WG3  O correction (rescale by alpha when the running max moves) and the
-//        epilogue (final reciprocal, BF16 store).
-// Tensor memory (512 columns allocated): S0 [0,128) S1 [128,256) O [256,384)
-// P0 [384,416) P1 [416,448).  FP32 scores of key tile j go to S(j%2) and its E4M3
-// probabilities (128 x 128 bytes = 32 columns) to P(j%2).  The softmax frees
-// S(j%2) as soon as it has read the scores, so QK(j+2) runs on the tensor
-// cores while the softmax of tile j is still computing; it writes P(j%2)
-// only after PV(j-2) has consumed the previous contents.
+//                 waits behind the other's dependencies.
+//   WG1  softmax of Q tile A, WG2 softmax of Q tile B; thread = one Q row, over
+//        every key tile in order.  Each warpgroup owns the whole running max
+//        and row sum of its rows, so the two never wait for each other and
+//        their exp2 phases (bound by the MUFU unit) drift apart instead of
+//        running side by side.
+//   WG3  O correction of both tiles (rescale by alpha when the running max
+//        moves) and the epilogue (final reciprocal, BF16 store).
+// Tensor memory (512 columns allocated): S(A) [0,128) S(B) [128,256)
+// O(A) [256,384) O(B) [384,512).  The softmax frees S(x) as soon as it has
+// read the scores, so QK of the next key tile runs on the tensor cores while
+// the softmax of this one is still computing.  Its E4M3 probabilities (128 x
+// 128 bytes) go to shared memory in the 128-byte-swizzled K-major layout the
+// PV MMA reads, once PV of the previous key tile has consumed the buffer.
 //
-// Every hand-off whose producer could otherwise run two phases ahead of its
-// consumer uses two barriers (indexed by key tile parity).  Every wait is
-// bounded: after the limit the waiter records H3ATTN_ERR_TIMEOUT in the
-// workspace status word, raises a CTA-wide abort flag, drains the
-// asynchronous work it issued and leaves; the tensor memory is freed.
+// Every wait is bounded: after the limit the waiter records
+// H3ATTN_ERR_TIMEOUT in the workspace status word, raises a CTA-wide abort
+// flag, drains the asynchronous work it issued and leaves; the tensor memory
+// is freed.  The barrier protocol is listed beside AttnSmem.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -49,12 +49,13 @@
 namespace h3 {
 namespace {
 
-constexpr int kStagesK = 3;  // K ring (BF16 tiles, 32 KB each)
-constexpr int kStagesV = 4;  // V ring (E4M3 tiles, 16 KB each)
+constexpr int kStagesK = 2;  // K ring (BF16 tiles, 32 KB each), shared by both Q tiles
+constexpr int kStagesV = 3;  // V ring (E4M3 tiles, 16 KB each)
 constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = 128 * 128;          // one 128 x 128-byte swizzled tile
 constexpr uint32_t kQKTileBytes = 2 * kTileBytes;   // a BF16 128 x 128 tile: two 64-column halves
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 416;
+__device__ __forceinline__ uint32_t col_s(int x) { return 128u * (uint32_t)x; }        // S(A), S(B)
+__device__ __forceinline__ uint32_t col_o(int x) { return 256u + 128u * (uint32_t)x; } // O(A), O(B)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
@@ -64,34 +65,52 @@ constexpr int64_t kRegSplitTotal = 128 * (kRegsControl + kRegsCorrection + 2 * k
 static_assert(kRegSplitTotal <= 65536, "register split exceeds the SM register file");
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 
+// Barrier protocol, per Q tile x and key tile j (phase j of each barrier unless
+// noted).  Each waiter is shown the back-edge that keeps its producer from
+// completing a later phase before the wait has been satisfied:
+//   s_full[x]   QK(x,j) done -> softmax x.   QK(x,j+1) needs s_free[x](j).
+//   s_free[x]   softmax x read S(x,j) -> QK issuer.  softmax x reaches the next
+//               arrival only after s_full[x](j+1), which needs this wait.
+//   m_full[x][j%2]  running max of tile j -> correction.  softmax x publishes
+//               m(j+2) only after pv_done[x](j) (P buffer), i.e. after the
+//               correction's o_ready[x](j), which follows its read of m(j).
+//   o_ready[x]  correction -> PV issuer.  The correction waits pv_done[x](j-1)
+//               before arriving for tile j, so phase j-1 has been consumed.
+//   p_full[x]   P(x,j) in shared memory -> PV issuer.  softmax x writes P(x,j+1)
+//               only after pv_done[x](j), i.e. after PV(x,j) was issued.
+//   pv_done[x]  PV(x,j) done -> softmax x (P buffer free) and correction (O
+//               final up to tile j).  PV(x,j+1) needs p_full[x](j+1) and
+//               o_ready[x](j+1), which both follow these waits.
+//   tok[A]      A's exp2 pass of tile j done -> softmax B (waits phase j).  A's
+//               pass of j+1 needs tok[B](j), which B arrives after this wait.
+//   tok[B]      B's exp2 pass of tile j done -> softmax A (waits phase j before
+//               its pass of j+1).  B's pass of j+1 needs tok[A](j+1), after it.
 struct __align__(1024) AttnSmem {
-  uint8_t q[2][kTileBytes];            // BF16 Q tile: key dims [0,64) and [64,128)
+  uint8_t q[2][2][kTileBytes];         // [Q tile][half] BF16 Q tiles: key dims [0,64) and [64,128)
   uint8_t k[kStagesK][2][kTileBytes];  // BF16 K tiles, same split
   uint8_t v[kStagesV][kTileBytes];     // E4M3 V^T tiles
+  uint8_t p[2][kTileBytes];            // [Q tile] E4M3 probabilities, SW128 K-major (A operand of PV)
   uint64_t q_full;
   uint64_t k_full[kStagesK], k_empty[kStagesK];
   uint64_t v_full[kStagesV], v_empty[kStagesV];
-  uint64_t s_full[2];   // MMA -> softmax: scores of key tile j in S(j%2)
-  uint64_t s_free[2];   // softmax -> MMA: scores of key tile j read, S(j%2) may be overwritten
-  uint64_t p_full[2];   // softmax -> MMA: P of key tile j in P(j%2)
-  uint64_t m_full[4];   // softmax of tile j -> softmax of tile j+1 and correction: running max in mrow[j%4]
-  uint64_t o_ready[2];  // correction -> MMA: O rescaled for key tile j
-  uint64_t pv_done[2];  // MMA -> correction, softmax: PV of key tile j completed (P(j%2) free)
-  uint64_t o_full;      // MMA -> epilogue: the last PV completed
-  uint64_t d_full;      // softmax (both warpgroups) -> epilogue: partial row sums published
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], o_ready[2];
+  uint64_t m_full[2][2];
+  uint64_t tok[2];    // [Q tile] softmax x finished its exp2 pass of key tile j (MUFU turn)
+  uint64_t o_full;    // MMA -> epilogue: the last PV completed
+  uint64_t d_full;    // softmax (both warpgroups) -> epilogue: row sums published
   uint64_t drain[2];  // QK issuer, PV issuer: all own MMAs completed
   uint32_t tmem_base;
   int abort;
   float sv[kD];
-  float mrow[4][kTile];   // [key tile % 4][row]: running max after that tile (log2 domain)
-  float dsum[2][kTile];   // [warpgroup][row]: sum of 448*p over its tiles, relative to mlast
-  float mlast[2][kTile];  // [warpgroup][row]: running max at its last tile
+  float mrow[2][2][kTile];  // [Q tile][key tile % 2][row]: running max after that tile (log2 domain)
+  float dsum[2][kTile];     // [Q tile][row]: sum of 448*p relative to the final max
 };
+static_assert(sizeof(AttnSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
 
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
-  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi
+  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi, kSiteSoftTok
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
@@ -111,7 +130,7 @@ constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23: float + magic rounds to a
 constexpr float kLog2_448 = 8.80735492205760410749f;
 // Key pairs, out of every 8, whose exp2 runs on the FMA pipe instead of MUFU.
 #ifndef H3ATTN_FMA_EXP2_PAIRS_OF_8
-#define H3ATTN_FMA_EXP2_PAIRS_OF_8 2
+#define H3ATTN_FMA_EXP2_PAIRS_OF_8 0
 #endif
 constexpr int kFmaExp2PairsOf8 = H3ATTN_FMA_EXP2_PAIRS_OF_8;
 
@@ -163,17 +182,14 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
   q1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
 }
 
-__device__ __forceinline__ float exp2_fma(float u) {
-  float q0, q1;
-  exp2_fma_pair(f2_pack(u, u), q0, q1);
-  return q0;
-}
 
-// Scaled probabilities of the 128 keys of a row: q = 2^(acc*f - mq) with
+// Scaled probabilities of the 128 keys of a row: q = 2^(s*f - mq) with
 // mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
 // into acc2 and the E4M3 words of q into w (4 keys per word).  kFmaExp2PairsOf8
 // key pairs in every eight take their exp2 from the FMA pipe (exp2_fma_pair),
-// the rest from MUFU, to balance the two units.
+// the rest from MUFU.  The exp2 is volatile so that it stays after the MUFU
+// turn's wait; the FMA, add and conversion work around it fills the MUFU
+// latency.
 template <bool kMasked>
 __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
                                          uint64_t (&acc2)[4], uint32_t (&w)[32]) {
@@ -193,8 +209,8 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
       } else {
         float u0, u1;
         f2_unpack(u, u0, u1);
-        q0 = ex2_ftz(u0);
-        q1 = ex2_ftz(u1);
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(u0));
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(u1));
       }
       if (kMasked) {
         if (i >= valid) q0 = 0.0f;
@@ -218,21 +234,21 @@ __device__ __forceinline__ void attn_teardown(uint32_t tmem, bool owner) {
 }
 
 // Timeline trace (debug export only): clock64() of per-key-tile events of one CTA,
-// trace[(event * 2 + slot) * nkv + j]; slot = key half for the softmax events, 0 otherwise.
+// trace[(event * 2 + slot) * nkv + j]; slot = Q tile (0 = A, 1 = B) of the pair.
 enum : int {
   kEvSReady = 0,   // softmax warp: scores of key tile j ready (after the wait)
-  kEvAlpha = 1,    // softmax warp: row maximum exchanged, alpha known
+  kEvMPub = 1,     // softmax warp: running max of tile j published to the correction
   kEvPDone = 2,    // softmax warp: probabilities stored, MMA issuer signalled
   kEvQK = 3,       // MMA issuer: QK of key tile j issued
-  kEvPV = 4,       // MMA issuer: P and O ready, PV of key tile j issued
-  kEvCorr = 5,     // correction warp: O rescaled (or skipped), MMA issuer signalled
-  kEvKFull = 6,    // MMA issuer: K tile j landed in shared memory
-  kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed (before the P store)
+  kEvPV = 4,       // MMA issuer: PV of key tile j issued
+  kEvCorr = 5,     // correction warp: O rescaled (or left alone), MMA issuer signalled
+  kEvKFull = 6,    // MMA issuer: K tile j landed in shared memory (slot 0)
+  kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed
   kEvPVDone = 8,   // MMA issuer: PV of key tile j issued and committed
-  kEvSFree = 9,    // MMA issuer: scores of key tile j released by the softmax (QK(j+2) may start)
+  kEvSFree = 9,    // MMA issuer: scores of key tile j released (QK of tile j+1 may start)
   kEvLd = 10,      // softmax warp: scores in registers
-  kEvMax = 11,     // softmax warp: own row maxima known (before the running-max hand-off)
-  kEvMWait = 12,   // softmax warp: running max of tile j-1 received
+  kEvMax = 11,     // softmax warp: own row maxima known
+  kEvPFree = 12,   // softmax warp: probability buffer free (PV of tile j-1 completed)
   kEvPVP = 13,     // MMA issuer: probabilities of key tile j observed (p_full)
   kEvPVO = 14,     // MMA issuer: O ready for key tile j observed (o_ready)
   kEvPDoneLast = 15,  // softmax warp of the last row quarter: probabilities handed over
@@ -264,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2, quarter = warp & 3;
   const int64_t h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
-  const int qt = blockIdx.x;  // Q tile index
+  const int qt0 = 2 * blockIdx.x;  // Q tiles qt0 (A) and qt0 + 1 (B)
+  const int nqt = (int)(p.Tq_pad / kTile);
   const int nkv = (p.Tkv + kTile - 1) / kTile;
   volatile int* abort = &sm.abort;
   const bool tracing =
@@ -284,15 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], kTile);
-      mbar_init(&sm.pv_done[i], 1);
-      mbar_init(&sm.p_full[i], kTile);
-      mbar_init(&sm.m_full[i], kTile);
-      mbar_init(&sm.m_full[i + 2], kTile);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.s_free[x], kTile);
+      mbar_init(&sm.p_full[x], kTile);
+      mbar_init(&sm.pv_done[x], 1);
+      mbar_init(&sm.o_ready[x], kTile);
+      mbar_init(&sm.m_full[x][0], kTile);
+      mbar_init(&sm.m_full[x][1], kTile);
+      mbar_init(&sm.tok[x], kTile);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&sm.o_ready[i], kTile);
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.d_full, 2 * kTile);
     mbar_init(&sm.drain[0], 1);
@@ -323,10 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        const int qrow = (int)(bh * p.Tq_pad + (int64_t)qt * kTile);
-        mbar_arrive_expect_tx(&sm.q_full, kQKTileBytes);
-        tma_load_2d(sm.q[0], &tm_q, &sm.q_full, 0, qrow);
-        tma_load_2d(sm.q[1], &tm_q, &sm.q_full, 64, qrow);
+        // Rows of Q tile B past this head's padded length (an odd tile count)
+        // are read from the next head or zero-filled; they are never stored.
+        mbar_arrive_expect_tx(&sm.q_full, 2 * kQKTileBytes);
+        for (int x = 0; x < 2; ++x) {
+          const int qrow = (int)(bh * p.Tq_pad + (int64_t)(qt0 + x) * kTile);
+          tma_load_2d(sm.q[x][0], &tm_q, &sm.q_full, 0, qrow);
+          tma_load_2d(sm.q[x][1], &tm_q, &sm.q_full, 64, qrow);
+        }
         const int krow = (int)(bh * p.Tkv_pad);
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
@@ -378,34 +400,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStagesK;
-          if (j >= 2) {
-            // S(j%2) is free once the softmax of tile j-2 has read its scores
-            if (!mbar_wait(&sm.s_free[j & 1], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs)) {
-              record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaS, abort);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            trace(kEvSFree, 0, j - 2);
-          }
           if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStagesK) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
             ok = false;
             break;
           }
-          tc_fence_after();
           trace(kEvKFull, 0, j);
-          const uint32_t s_col = (j & 1) ? kColS1 : kColS0;
-          // 8 MMAs of K = 16: BF16 key dims [16kk, 16kk+16) = bytes 32*(kk%4) of half kk/4
+          for (int x = 0; x < 2; ++x) {
+            if (j >= 1) {
+              // S(x) is free once the softmax of Q tile x has read key tile j-1
+              if (!mbar_wait(&sm.s_free[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs)) {
+                record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaS, abort);
+                ok = false;
+                break;
+              }
+              trace(kEvSFree, x, j - 1);
+            }
+            tc_fence_after();
+            // 8 MMAs of K = 16: BF16 key dims [16kk, 16kk+16) = bytes 32*(kk%4) of half kk/4
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q[kk >> 2])) + 2 * (kk & 3);
-            const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s][kk >> 2])) + 2 * (kk & 3);
-            mma_bf16_ss(tmem + s_col, dq, dk, kIdescQK, kk > 0);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t dq = sdesc_k_sw128(smem_u32(sm.q[x][kk >> 2])) + 2 * (kk & 3);
+              const uint64_t dk = sdesc_k_sw128(smem_u32(sm.k[s][kk >> 2])) + 2 * (kk & 3);
+              mma_bf16_ss(tmem + col_s(x), dq, dk, kIdescQK, kk > 0);
+            }
+            mma_commit(&sm.s_full[x]);
+            trace(kEvQK, x, j);
           }
-          mma_commit(&sm.s_full[j & 1]);
+          if (!ok) break;
           mma_commit(&sm.k_empty[s]);
-          trace(kEvQK, 0, j);
         }
         // wait until every MMA this thread issued has completed
         mma_commit(&sm.drain[0]);
@@ -418,33 +441,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStagesV;
-          if (!mbar_wait(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
-            ok = false;
-            break;
-          }
-          trace(kEvPVP, 0, j);
-          if (!mbar_wait(&sm.o_ready[j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs)) {
-            record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
-            ok = false;
-            break;
-          }
-          trace(kEvPVO, 0, j);
           if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStagesV) & 1u, abort, kWaitLimitNs)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaV, abort);
             ok = false;
             break;
           }
-          tc_fence_after();
-          trace(kEvPV, 0, j);
           const uint64_t dv = sdesc_k_sw128(smem_u32(sm.v[s]));
-          const uint32_t p_col = (j & 1) ? kColP1 : kColP0;
+          for (int x = 0; x < 2; ++x) {
+            if (!mbar_wait(&sm.p_full[x], (uint32_t)j & 1u, abort, kWaitLimitNs)) {
+              record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
+              ok = false;
+              break;
+            }
+            trace(kEvPVP, x, j);
+            if (!mbar_wait(&sm.o_ready[x], (uint32_t)j & 1u, abort, kWaitLimitNs)) {
+              record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
+              ok = false;
+              break;
+            }
+            trace(kEvPVO, x, j);
+            tc_fence_after();
+            trace(kEvPV, x, j);
+            const uint64_t dp = sdesc_k_sw128(smem_u32(sm.p[x]));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts(tmem + kColO, tmem + p_col + 8 * kk, dv + 2 * kk, kIdescPV, j > 0 || kk > 0);
-          mma_commit(&sm.pv_done[j & 1]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8_ss(tmem + col_o(x), dp + 2 * kk, dv + 2 * kk, kIdescPV, j > 0 || kk > 0);
+            mma_commit(&sm.pv_done[x]);
+            trace(kEvPVDone, x, j);
+          }
+          if (!ok) break;
           mma_commit(&sm.v_empty[s]);
-          trace(kEvPVDone, 0, j);
         }
         if (ok) mma_commit(&sm.o_full);
         mma_commit(&sm.drain[1]);
@@ -460,57 +486,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (wg == 3) {
     // -------------------------------------------- correction + epilogue ----
     regs_dealloc<kRegsCorrection>();
-    const uint32_t tO = tmem_lane_addr(tmem, quarter, kColO);
     bool ok = true;
-    float m_prev = -INFINITY;  // running max after key tile j-1
-    for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(&sm.m_full[j & 3], (uint32_t)(j >> 2) & 1u, abort, kWaitLimitNs);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) {
-        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrM, abort);
-        break;
-      }
-      const float m_j = sm.mrow[j & 3][row];
-      const float alpha = ex2_approx(__fsub_rn(m_prev, m_j));
-      m_prev = m_j;
-      if (j > 0) {
-        // A warp whose rows all kept their maximum leaves O alone: PV(j) may follow
-        // PV(j-1) in the tensor pipe directly.  It still waits for PV(j-2), which
-        // consumed the previous phase of o_ready[j%2], so that this warpgroup never
-        // runs two phases ahead of the PV issuer.  A warp that rescales needs O to
-        // hold the sum over key tiles < j, i.e. PV(j-1) completed.
-        const bool rescale = __any_sync(0xFFFFFFFFu, alpha != 1.0f);
-        const int jw = rescale ? j - 1 : j - 2;
-        if (jw >= 0) {
-          ok = mbar_wait(&sm.pv_done[jw & 1], (uint32_t)(jw >> 1) & 1u, abort, kWaitLimitNs);
+    float m_prev[2] = {-INFINITY, -INFINITY};  // running max of each Q tile after key tile j-1
+    for (int j = 0; ok && j < nkv; ++j) {
+      for (int x = 0; x < 2; ++x) {
+        ok = mbar_wait(&sm.m_full[x][j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrM, abort);
+          break;
+        }
+        const float m_j = sm.mrow[x][j & 1][row];
+        const float alpha = ex2_approx(__fsub_rn(m_prev[x], m_j));
+        m_prev[x] = m_j;
+        if (j > 0) {
+          // O(x) holds the sum over key tiles < j once PV(x, j-1) has completed;
+          // the wait also retires the previous phase of o_ready[x].
+          ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs);
           ok = __all_sync(0xFFFFFFFFu, ok);
           if (!ok) {
             if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
             break;
           }
-        }
-        if (rescale) {
-          tc_fence_after();
-          const uint64_t aa = f2_pack(alpha, alpha);
+          if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+            tc_fence_after();
+            const uint32_t tO = tmem_lane_addr(tmem, quarter, col_o(x));
+            const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * ch, o);
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * ch, o);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
-              o[e] = __float_as_uint(lo);
-              o[e + 1] = __float_as_uint(hi);
+              for (int e = 0; e < 32; e += 2) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), aa), lo, hi);
+                o[e] = __float_as_uint(lo);
+                o[e + 1] = __float_as_uint(hi);
+              }
+              tmem_st32(tO + 32 * ch, o);
             }
-            tmem_st32(tO + 32 * ch, o);
+            tmem_wait_st();
           }
-          tmem_wait_st();
         }
+        tc_fence_before();
+        mbar_arrive(&sm.o_ready[x]);
+        if (quarter == 0 && lane == 0) trace(kEvCorr, x, j);
       }
-      tc_fence_before();
-      mbar_arrive(&sm.o_ready[j & 1]);
-      if (quarter == 0 && lane == 0) trace(kEvCorr, 0, j);
     }
     if (ok) {
       ok = mbar_wait(&sm.d_full, 0, abort, kWaitLimitNs) && mbar_wait(&sm.o_full, 0, abort, kWaitLimitNs);
@@ -519,31 +540,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      // d = sum over tiles of 448*p relative to the final max, from the two warpgroups
-      const float m0 = sm.mlast[0][row], m1 = sm.mlast[1][row];
-      const float mf = fmaxf(m0, m1);
-      const float d = __fadd_rn(__fmul_rn(sm.dsum[0][row], ex2_approx(__fsub_rn(m0, mf))),
-                                __fmul_rn(sm.dsum[1][row], ex2_approx(__fsub_rn(m1, mf))));
-      const float r = __frcp_rn(d);
-      const int64_t grow = (int64_t)qt * kTile + row;
-      __nv_bfloat16* orow = p.out + b * p.out_sb + grow * p.out_st + h * p.out_sh;
+      for (int x = 0; x < 2; ++x) {
+        // d = sum over key tiles of 448*p relative to the final max
+        const float r = __frcp_rn(sm.dsum[x][row]);
+        const int64_t grow = (int64_t)(qt0 + x) * kTile + row;
+        const uint32_t tO = tmem_lane_addr(tmem, quarter, col_o(x));
+        __nv_bfloat16* orow = p.out + b * p.out_sb + grow * p.out_st + h * p.out_sh;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * ch, o);
-        if (grow < p.Tq) {
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * ch, o);
+          if (grow < p.Tq) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t w[4];
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t w[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int c0 = 32 * ch + e + 2 * u;
-              const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u]), r), sm.sv[c0]);
-              const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u + 1]), r), sm.sv[c0 + 1]);
-              const __nv_bfloat162 pr2 = __floats2bfloat162_rn(y0, y1);
-              w[u] = *reinterpret_cast<const uint32_t*>(&pr2);
+              for (int u = 0; u < 4; ++u) {
+                const int c0 = 32 * ch + e + 2 * u;
+                const float y0 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u]), r), sm.sv[c0]);
+                const float y1 = __fmul_rn(__fmul_rn(__uint_as_float(o[e + 2 * u + 1]), r), sm.sv[c0 + 1]);
+                const __nv_bfloat162 pr2 = __floats2bfloat162_rn(y0, y1);
+                w[u] = *reinterpret_cast<const uint32_t*>(&pr2);
+              }
+              *reinterpret_cast<uint4*>(orow + 32 * ch + e) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            *reinterpret_cast<uint4*>(orow + 32 * ch + e) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -554,27 +574,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // -------------------------------------------------------- softmax ----
   regs_alloc<kRegsSoftmax>();
-  const int par = wg - 1;  // this warpgroup owns key tiles j with j % 2 == par (scores in S(par))
+  const int x = wg - 1;  // this warpgroup owns Q tile x of the pair, over all key tiles
   {
-    const float sqi = p.sq[bh * (p.Tq_pad / kQGroup) + (int64_t)qt * (kTile / kQGroup) + quarter];
+    // a Q tile past the padded length (odd tile count) reuses the last tile's scale
+    const int qts = min(qt0 + x, nqt - 1);
+    const float sqi = p.sq[bh * (p.Tq_pad / kQGroup) + (int64_t)qts * (kTile / kQGroup) + quarter];
     const float* skh = p.sk + bh * (p.Tkv_pad / kKGroup);
-    const uint32_t tS = tmem_lane_addr(tmem, quarter, par ? kColS1 : kColS0);
-    const uint32_t tP = tmem_lane_addr(tmem, quarter, par ? kColP1 : kColP0);
-    float m_w = -INFINITY, d_w = 0.0f;  // running max at this warpgroup's previous tile, its sum
-    float sk0 = 0.0f, sk1 = 0.0f;
-    if (par < nkv) {
-      sk0 = __ldg(skh + 2 * par);
-      sk1 = __ldg(skh + 2 * par + 1);
-    }
+    const uint32_t tS = tmem_lane_addr(tmem, quarter, col_s(x));
+    // this row of the swizzled probability tile: 16-byte chunk c at c ^ (row % 8)
+    const uint32_t prow = smem_u32(sm.p[x]) + (uint32_t)row * 128u;
+    float m_w = -INFINITY, d_w = 0.0f;  // running max after the previous key tile, its row sum
+    float sk0 = __ldg(skh), sk1 = __ldg(skh + 1);
     bool ok = true;
-    for (int j = par; j < nkv; j += 2) {
+    for (int j = 0; j < nkv; ++j) {
       const float f0 = __fmul_rn(__fmul_rn(sqi, sk0), p.c_log2);
       const float f1 = __fmul_rn(__fmul_rn(sqi, sk1), p.c_log2);
-      if (j + 2 < nkv) {
-        sk0 = __ldg(skh + 2 * (j + 2));
-        sk1 = __ldg(skh + 2 * (j + 2) + 1);
+      if (j + 1 < nkv) {
+        sk0 = __ldg(skh + 2 * (j + 1));
+        sk1 = __ldg(skh + 2 * (j + 1) + 1);
       }
-      ok = mbar_wait(&sm.s_full[par], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
+      ok = mbar_wait(&sm.s_full[x], (uint32_t)j & 1u, abort, kWaitLimitNs);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
         if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
@@ -582,76 +601,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const bool tr = kTrace && tracing && quarter == 0 && lane == 0;
-      if (tr) trace(kEvSReady, par, j);
+      if (tr) trace(kEvSReady, x, j);
       const int valid = min(kTile, p.Tkv - j * kTile);
-      uint32_t x[128];
-      tmem_ld64x2(tS, x);
+      uint32_t xs[128];
+      tmem_ld64x2(tS, xs);
       tc_fence_before();
-      mbar_arrive(&sm.s_free[par]);
-      if (tr) trace(kEvLd, par, j);
+      mbar_arrive(&sm.s_free[x]);
+      if (tr) trace(kEvLd, x, j);
       float xm0, xm1;
       if (valid < kTile)
-        rowmax128<true>(x, valid, xm0, xm1);
+        rowmax128<true>(xs, valid, xm0, xm1);
       else
-        rowmax128<false>(x, valid, xm0, xm1);
+        rowmax128<false>(xs, valid, xm0, xm1);
       const float t0m = __fmul_rn(xm0, f0);  // valid >= 1: half 0 has a key
       const float t1m = valid > 64 ? __fmul_rn(xm1, f1) : -INFINITY;
       if (tr) {
         asm volatile("" ::"f"(t0m), "f"(t1m));  // the maxima exist before the stamp is taken
-        trace(kEvMax, par, j);
+        trace(kEvMax, x, j);
       }
-      // running max after tile j-1, from the other warpgroup
-      float m_prev = -INFINITY;
-      if (j > 0) {
-        ok = mbar_wait(&sm.m_full[(j - 1) & 3], (uint32_t)((j - 1) >> 2) & 1u, abort, kWaitLimitNs);
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (!ok) {
-          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftM, abort);
-          break;
-        }
-        m_prev = sm.mrow[(j - 1) & 3][row];
-      }
-      if (tr) trace(kEvMWait, par, j);
-      const float m_j = fmaxf(m_prev, fmaxf(t0m, t1m));
-      sm.mrow[j & 3][row] = m_j;
-      mbar_arrive(&sm.m_full[j & 3]);
-      if (tr) trace(kEvAlpha, par, j);
+      const float m_j = fmaxf(m_w, fmaxf(t0m, t1m));
+      sm.mrow[x][j & 1][row] = m_j;
+      mbar_arrive(&sm.m_full[x][j & 1]);
+      if (tr) trace(kEvMPub, x, j);
       uint32_t pw[32];
       uint64_t acc2[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
       const float mq = __fsub_rn(m_j, kLog2_448);
+      // MUFU turn: the exp2 passes alternate A(0) B(0) A(1) B(1) ... so that
+      // each runs with the MUFU unit to itself while the other warpgroup does
+      // the rest of its tile.
+      if (x == 1 || j >= 1) {
+        const int jt = x == 1 ? j : j - 1;  // A waits for B's pass of j-1, B for A's pass of j
+        ok = mbar_wait(&sm.tok[1 - x], (uint32_t)jt & 1u, abort, kWaitLimitNs);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftTok, abort);
+          break;
+        }
+      }
       if (valid < kTile)
-        probs128<true>(x, valid, f0, f1, mq, acc2, pw);
+        probs128<true>(xs, valid, f0, f1, mq, acc2, pw);
       else
-        probs128<false>(x, valid, f0, f1, mq, acc2, pw);
-      if (tr) trace(kEvProbs, par, j);
-      if (j >= 2) {
-        // P(j%2) still feeds PV(j-2) until that MMA has completed
-        ok = mbar_wait(&sm.pv_done[par], (uint32_t)((j - 2) >> 1) & 1u, abort, kWaitLimitNs);
+        probs128<false>(xs, valid, f0, f1, mq, acc2, pw);
+      mbar_arrive(&sm.tok[x]);
+      if (tr) trace(kEvProbs, x, j);
+      if (j >= 1) {
+        // the probability buffer still feeds PV(x, j-1) until that MMA has completed
+        ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftPV, abort);
           break;
         }
-        tc_fence_after();
+        if (tr) trace(kEvPFree, x, j);
       }
-      tmem_st32(tP, pw);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.p_full[par]);
-      if (tr) trace(kEvPDone, par, j);
-      if (kTrace && tracing && quarter == 3 && lane == 0) trace(kEvPDoneLast, par, j);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + ((uint32_t)(c ^ (row & 7)) << 4)),
+                     "r"(pw[4 * c]), "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3])
+                     : "memory");
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.p_full[x]);
+      if (tr) trace(kEvPDone, x, j);
+      if (kTrace && tracing && quarter == 3 && lane == 0) trace(kEvPDoneLast, x, j);
       float a[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
       const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-      d_w = __fadd_rn(__fmul_rn(d_w, exp2_fma(__fsub_rn(m_w, m_j))), es);
+      d_w = __fadd_rn(__fmul_rn(d_w, ex2_approx(__fsub_rn(m_w, m_j))), es);
       m_w = m_j;
     }
     if (ok) {
-      sm.dsum[par][row] = d_w;
-      sm.mlast[par][row] = m_w;
+      sm.dsum[x][row] = d_w;
       mbar_arrive(&sm.d_full);
     }
   }
@@ -828,7 +850,7 @@ cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, fl
   p.status = reinterpret_cast<DevStatus*>(const_cast<char*>(ws) + L.off[H3ATTN_WS_STATUS]);
   p.trace = trace;
   p.trace_block = trace_block;
-  dim3 grid((unsigned)(s.Tq_pad / kTile), (unsigned)s.H, (unsigned)s.B);
+  dim3 grid((unsigned)((s.Tq_pad / kTile + 1) / 2), (unsigned)s.H, (unsigned)s.B);
   if (trace != nullptr)
     attn_sm100_kernel<true><<<grid, kThreads, kAttnSmemBytes, st>>>(tq, tk, tv, p);
   else

@@ -70,7 +70,9 @@ struct DevStatus {
 cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
                             const Shape& s, const Layout& L, char* ws, cudaStream_t st);
 
-struct TmapSet;  // opaque; attention.cu
+// The attention grid: one CTA per pair of 128-row Q tiles of one (b, h).
+inline int64_t attention_ctas(const Shape& s) { return ((s.Tq_pad / kTile + 1) / 2) * (int64_t)s.H * s.B; }
+
 cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
                              const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why,
                              uint64_t* trace = nullptr, int trace_block = -1);

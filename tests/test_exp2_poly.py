@@ -1,9 +1,10 @@
 """The FMA-pipe exp2 of the attention kernel against the exact 2^u (an error bound).
 
-The kernel evaluates a quarter of its probabilities without the MUFU unit:
-n = rint(u) through the 1.5*2^23 magic number, r = u - n, 2^r by a degree-5
-polynomial in FP32 Horner form (one rounding per fused multiply-add), then n
-added into the exponent field.  This test reads the coefficients the kernel is
+Built with H3ATTN_FMA_EXP2_PAIRS_OF_8=k (k of every 8 key pairs; 0 by default,
+where every probability comes from MUFU), the kernel evaluates part of its
+probabilities without the MUFU unit: n = rint(u) through the 1.5*2^23 magic
+number, r = u - n, 2^r by a degree-5 polynomial in FP32 Horner form (one
+rounding per fused multiply-add), then n added into the exponent field.  This test reads the coefficients the kernel is
 built with (csrc/exp2_poly.h), replays those exact FP32 steps in numpy and
 checks the result against 2^u in FP64 over the argument range the kernel
 produces (u in [-125, log2(448)]).  The bound it enforces, 2.5e-7 relative, is
