@@ -143,8 +143,25 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
                                      int D, int b, int h, int qt, int kt, int32_t* out_dev,
                                      void* stream);
 
+/* Failure-path test hook: h3attn_attend with every barrier wait bounded by
+ * wait_limit_ns (1 ms to 2 s) and the correction warpgroup's "O ready" arrivals
+ * withheld, so that the PV issuer's wait, and every wait behind it, has no
+ * producer.  The first of them to run out records H3ATTN_ERR_TIMEOUT in the
+ * workspace status word (detail word: its wait-site id; block word: its CTA),
+ * raises its CTA's abort flag, and every role of the CTA drains the copies and
+ * tensor-core work it started, frees the tensor memory and returns; no fault,
+ * trap or unbounded wait is involved, and the CUDA context stays usable.
+ * Returns H3ATTN_OK when the launch was made; h3attn_check_status then reports
+ * H3ATTN_ERR_TIMEOUT.  Output rows are unspecified.  Arguments as h3attn_attend.
+ * Tests the failure side of the no-deadlock requirement of "Phase 2B Aligned
+ * Numerical Prototype", Exactness: a wait whose producer never arrives ends with
+ * an error status instead of a hang. */
+h3attn_status h3attn_debug_attend_timeout(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H,
+                                          int D, float softmax_scale, const h3attn_bf16_out* out,
+                                          uint64_t wait_limit_ns, void* stream);
+
 /* Tracing export: h3attn_attend with a timeline probe in one CTA (linear block index
- * trace_block; CTAs are (Q tile, head, batch), Q tile fastest).  Writes clock64()
+ * trace_block; CTAs are (pair of 128-row Q tiles, head, batch), pair fastest).  Writes clock64()
  * stamps of 16 events for each key tile j to trace_dev[(event*2 + slot)*ceil(Tkv/128) + j]
  * (uint64, device memory, 32*ceil(Tkv/128) entries; entries of events that did not
  * happen are left untouched).  Softmax events use slot = j % 2 (the warpgroup that owns

@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.h3attn_debug_qk_scores.argtypes = [P, S] + [I] * 9 + [P, P]
         L.h3attn_debug_attend_trace.restype = I
         L.h3attn_debug_attend_trace.argtypes = [P, S] + [I] * 5 + [F, VP, I, P, P]
+        L.h3attn_debug_attend_timeout.restype = I
+        L.h3attn_debug_attend_timeout.argtypes = [P, S] + [I] * 5 + [F, VP, ctypes.c_uint64, P]
         L.h3attn_status_string.restype = ctypes.c_char_p
         L.h3attn_status_string.argtypes = [I]
         L.h3attn_version.restype = I
@@ -207,6 +209,16 @@ def h3attn_debug_attend_trace(ws, B: int, Tq: int, Tkv: int, H: int, softmax_sca
                                            tr.data_ptr(), _stream(stream)), "h3attn_debug_attend_trace")
     t = tr.view(len(TRACE_EVENTS), 2, nkv).cpu()
     return {name: t[i] for i, name in enumerate(TRACE_EVENTS)}
+
+
+def h3attn_debug_attend_timeout(ws, B: int, Tq: int, Tkv: int, H: int, softmax_scale: float, out,
+                                wait_limit_ns: int, stream=None, D: int = HEAD_DIM):
+    """h3attn_attend with the correction's O-ready arrivals withheld and every wait bounded by
+    wait_limit_ns: the launch ends with H3ATTN_ERR_TIMEOUT in the workspace status word."""
+    wp, wb = _ptr_bytes(ws)
+    vo = _view(out)
+    _check(lib().h3attn_debug_attend_timeout(wp, wb, B, Tq, Tkv, H, D, softmax_scale, ctypes.byref(vo),
+                                             int(wait_limit_ns), _stream(stream)), "h3attn_debug_attend_timeout")
 
 
 def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:

@@ -171,6 +171,25 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
   return H3ATTN_OK;
 }
 
+h3attn_status h3attn_debug_attend_timeout(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H, int D,
+                                          float softmax_scale, const h3attn_bf16_out* out,
+                                          uint64_t wait_limit_ns, void* stream) {
+  H3_TRY(check_sizes(B, Tq, Tkv, H, D));
+  H3_TRY(check_out(out));
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return H3ATTN_ERR_INVALID_ARG;
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > kDefaultWaitLimitNs) return H3ATTN_ERR_INVALID_ARG;
+  const Shape s = make_shape(B, Tq, Tkv, H);
+  const Layout L = make_layout(s);
+  H3_TRY(check_ws(ws, ws_bytes, L));
+  H3_TRY(check_device());
+  const float c_log2 = (float)((double)softmax_scale * kLog2e);
+  h3attn_status why = H3ATTN_OK;
+  if (launch_attention(static_cast<const char*>(ws), s, L, c_log2, *out, static_cast<cudaStream_t>(stream), &why,
+                       nullptr, -1, wait_limit_ns, true) != cudaSuccess)
+    return why != H3ATTN_OK ? why : H3ATTN_ERR_CUDA;
+  return H3ATTN_OK;
+}
+
 h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H, int D,
                                         float softmax_scale, const h3attn_bf16_out* out, int trace_block,
                                         uint64_t* trace_dev, void* stream) {

@@ -58,7 +58,7 @@ __device__ __forceinline__ uint32_t col_s(int x) { return 128u * (uint32_t)x; } 
 __device__ __forceinline__ uint32_t col_o(int x) { return 256u + 128u * (uint32_t)x; } // O(A), O(B)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kWaitLimitNs = kDefaultWaitLimitNs;
 // setmaxnreg split (registers per thread): control, correction, softmax warpgroups.
 constexpr int kRegsControl = 64, kRegsCorrection = 56, kRegsSoftmax = 192;
 constexpr int64_t kRegSplitTotal = 128 * (kRegsControl + kRegsCorrection + 2 * kRegsSoftmax);
@@ -256,6 +256,12 @@ enum : int {
 };
 static_assert(kNumEvents == kTraceEvents, "trace buffer layout");
 
+// Failure-path test hook: with kWithholdOReady the correction warpgroup never
+// arrives on o_ready, so the PV issuer's first wait runs out after
+// wait_limit_ns; it records H3ATTN_ERR_TIMEOUT (site kSiteMmaO) and raises the
+// abort flag, and every other role leaves through its drain path.
+constexpr int kWithholdNone = 0, kWithholdOReady = 1;
+
 struct AttnParams {
   const float* sq;   // [B,H,Tq_pad/32]
   const float* sk;   // [B,H,Tkv_pad/64]
@@ -268,6 +274,8 @@ struct AttnParams {
   DevStatus* status;
   uint64_t* trace;   // timeline trace buffer (traced instantiation only)
   int trace_block;   // linear block index that records the trace
+  uint64_t wait_limit_ns;  // bound of every barrier wait
+  int withhold;      // test hook: kWithholdOReady makes the correction skip its o_ready arrivals
 };
 
 template <bool kTrace>
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
           const int s = j % kStagesK;
-          if (!mbar_wait(&sm.k_empty[s], ((uint32_t)(j / kStagesK) & 1u) ^ 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.k_empty[s], ((uint32_t)(j / kStagesK) & 1u) ^ 1u, abort, p.wait_limit_ns)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdKEmpty, abort);
             break;
           }
@@ -378,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
           const int s = j % kStagesV;
-          if (!mbar_wait(&sm.v_empty[s], ((uint32_t)(j / kStagesV) & 1u) ^ 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.v_empty[s], ((uint32_t)(j / kStagesV) & 1u) ^ 1u, abort, p.wait_limit_ns)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteProdVEmpty, abort);
             break;
           }
@@ -395,12 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------------ QK issuer ----
       if (lane == 0) {
-        bool ok = mbar_wait(&sm.q_full, 0, abort, kWaitLimitNs);
+        bool ok = mbar_wait(&sm.q_full, 0, abort, p.wait_limit_ns);
         if (!ok) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaQ, abort);
         tc_fence_after();
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStagesK;
-          if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStagesK) & 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.k_full[s], (uint32_t)(j / kStagesK) & 1u, abort, p.wait_limit_ns)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaK, abort);
             ok = false;
             break;
@@ -409,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 2; ++x) {
             if (j >= 1) {
               // S(x) is free once the softmax of Q tile x has read key tile j-1
-              if (!mbar_wait(&sm.s_free[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs)) {
+              if (!mbar_wait(&sm.s_free[x], (uint32_t)(j - 1) & 1u, abort, p.wait_limit_ns)) {
                 record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaS, abort);
                 ok = false;
                 break;
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // wait until every MMA this thread issued has completed
         mma_commit(&sm.drain[0]);
-        mbar_wait(&sm.drain[0], 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
+        mbar_wait(&sm.drain[0], 0, nullptr, ok ? p.wait_limit_ns : kDrainLimitNs);
       }
       __syncwarp();
     } else if (warp == 3) {
@@ -441,20 +449,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
           const int s = j % kStagesV;
-          if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStagesV) & 1u, abort, kWaitLimitNs)) {
+          if (!mbar_wait(&sm.v_full[s], (uint32_t)(j / kStagesV) & 1u, abort, p.wait_limit_ns)) {
             record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaV, abort);
             ok = false;
             break;
           }
           const uint64_t dv = sdesc_k_sw128(smem_u32(sm.v[s]));
           for (int x = 0; x < 2; ++x) {
-            if (!mbar_wait(&sm.p_full[x], (uint32_t)j & 1u, abort, kWaitLimitNs)) {
+            if (!mbar_wait(&sm.p_full[x], (uint32_t)j & 1u, abort, p.wait_limit_ns)) {
               record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaP, abort);
               ok = false;
               break;
             }
             trace(kEvPVP, x, j);
-            if (!mbar_wait(&sm.o_ready[x], (uint32_t)j & 1u, abort, kWaitLimitNs)) {
+            if (!mbar_wait(&sm.o_ready[x], (uint32_t)j & 1u, abort, p.wait_limit_ns)) {
               record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteMmaO, abort);
               ok = false;
               break;
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) mma_commit(&sm.o_full);
         mma_commit(&sm.drain[1]);
-        mbar_wait(&sm.drain[1], 0, nullptr, ok ? kWaitLimitNs : kDrainLimitNs);
+        mbar_wait(&sm.drain[1], 0, nullptr, ok ? p.wait_limit_ns : kDrainLimitNs);
       }
       __syncwarp();
     }
@@ -490,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_prev[2] = {-INFINITY, -INFINITY};  // running max of each Q tile after key tile j-1
     for (int j = 0; ok && j < nkv; ++j) {
       for (int x = 0; x < 2; ++x) {
-        ok = mbar_wait(&sm.m_full[x][j & 1], (uint32_t)(j >> 1) & 1u, abort, kWaitLimitNs);
+        ok = mbar_wait(&sm.m_full[x][j & 1], (uint32_t)(j >> 1) & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrM, abort);
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j > 0) {
           // O(x) holds the sum over key tiles < j once PV(x, j-1) has completed;
           // the wait also retires the previous phase of o_ready[x].
-          ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs);
+          ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, p.wait_limit_ns);
           ok = __all_sync(0xFFFFFFFFu, ok);
           if (!ok) {
             if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrPV, abort);
@@ -529,12 +537,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(&sm.o_ready[x]);
+        if (p.withhold != kWithholdOReady) mbar_arrive(&sm.o_ready[x]);
         if (quarter == 0 && lane == 0) trace(kEvCorr, x, j);
       }
     }
     if (ok) {
-      ok = mbar_wait(&sm.d_full, 0, abort, kWaitLimitNs) && mbar_wait(&sm.o_full, 0, abort, kWaitLimitNs);
+      ok = mbar_wait(&sm.d_full, 0, abort, p.wait_limit_ns) && mbar_wait(&sm.o_full, 0, abort, p.wait_limit_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok && lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteEpi, abort);
     }
@@ -593,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sk0 = __ldg(skh + 2 * (j + 1));
         sk1 = __ldg(skh + 2 * (j + 1) + 1);
       }
-      ok = mbar_wait(&sm.s_full[x], (uint32_t)j & 1u, abort, kWaitLimitNs);
+      ok = mbar_wait(&sm.s_full[x], (uint32_t)j & 1u, abort, p.wait_limit_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
         if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
@@ -633,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the rest of its tile.
       if (x == 1 || j >= 1) {
         const int jt = x == 1 ? j : j - 1;  // A waits for B's pass of j-1, B for A's pass of j
-        ok = mbar_wait(&sm.tok[1 - x], (uint32_t)jt & 1u, abort, kWaitLimitNs);
+        ok = mbar_wait(&sm.tok[1 - x], (uint32_t)jt & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftTok, abort);
@@ -648,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tr) trace(kEvProbs, x, j);
       if (j >= 1) {
         // the probability buffer still feeds PV(x, j-1) until that MMA has completed
-        ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, kWaitLimitNs);
+        ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftPV, abort);
@@ -821,7 +829,7 @@ cudaError_t ensure_attrs() {
 
 cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
                              const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why, uint64_t* trace,
-                             int trace_block) {
+                             int trace_block, uint64_t wait_limit_ns, bool withhold_o_ready) {
   *why = H3ATTN_OK;
   cudaError_t e = ensure_attrs();
   if (e != cudaSuccess) return e;
@@ -850,6 +858,8 @@ cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, fl
   p.status = reinterpret_cast<DevStatus*>(const_cast<char*>(ws) + L.off[H3ATTN_WS_STATUS]);
   p.trace = trace;
   p.trace_block = trace_block;
+  p.wait_limit_ns = wait_limit_ns;
+  p.withhold = withhold_o_ready ? kWithholdOReady : kWithholdNone;
   dim3 grid((unsigned)((s.Tq_pad / kTile + 1) / 2), (unsigned)s.H, (unsigned)s.B);
   if (trace != nullptr)
     attn_sm100_kernel<true><<<grid, kThreads, kAttnSmemBytes, st>>>(tq, tk, tv, p);

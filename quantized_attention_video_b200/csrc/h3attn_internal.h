@@ -73,9 +73,11 @@ cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k
 // The attention grid: one CTA per pair of 128-row Q tiles of one (b, h).
 inline int64_t attention_ctas(const Shape& s) { return ((s.Tq_pad / kTile + 1) / 2) * (int64_t)s.H * s.B; }
 
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // bound of every barrier wait: 2 s
 cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, float c_log2,
                              const h3attn_bf16_out& out, cudaStream_t st, h3attn_status* why,
-                             uint64_t* trace = nullptr, int trace_block = -1);
+                             uint64_t* trace = nullptr, int trace_block = -1,
+                             uint64_t wait_limit_ns = kDefaultWaitLimitNs, bool withhold_o_ready = false);
 constexpr int kTraceEvents = 16;  // events per (tile slot, key tile) in the timeline trace
 cudaError_t launch_debug_qk(const char* ws, const Shape& s, const Layout& L, int b, int h, int qt, int kt,
                             int32_t* out, cudaStream_t st, h3attn_status* why);
