@@ -322,8 +322,9 @@ def run_ours(args, w):
                 "algorithmic_ops_per_launch": ops,
                 "traffic": None if tr is None else tr["dram_bytes_per_launch_full"],
                 "quantize_ms": quant_avg, "attention_ms": attn_avg,
-                # stats reads K, V (4 B); quantize reads Q, K, V (2 + 4 B) and writes q8, k8, v8 (1 + 2 B)
-                "quantize_gbs": (10 * w.Tkv + 3 * w.Tq) * w.B * w.H * w.D / (quant_avg * 1e-3) / 1e9}
+                # stats reads K, V (4 B); quantize reads Q, K, V (2 + 4 B) and writes the Q, K words
+                # (2 + 2 B, INT8 values held as BF16) and v8 (1 B)
+                "quantize_gbs": (11 * w.Tkv + 4 * w.Tq) * w.B * w.H * w.D / (quant_avg * 1e-3) / 1e9}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
