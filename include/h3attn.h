@@ -164,16 +164,17 @@ h3attn_status h3attn_debug_attend_timeout(const void* ws, size_t ws_bytes, int B
  * trace_block; CTAs are (pair of 128-row Q tiles, head, batch), pair fastest).  Writes clock64()
  * stamps of 16 events for each key tile j to trace_dev[(event*2 + slot)*ceil(Tkv/128) + j]
  * (uint64, device memory, 32*ceil(Tkv/128) entries; entries of events that did not
- * happen are left untouched).  Softmax events use slot = j % 2 (the warpgroup that owns
- * tile j), the others slot 0.  Events: 0 scores ready in the softmax warp, 1 running max
- * of tile j published, 2 probabilities handed to the MMA issuer, 3 QK issued, 4 PV
- * issued, 5 O rescaled (or left alone) by the correction warp, 6 K tile landed,
- * 7 probabilities computed, 8 PV issued and committed, 9 scores released (the next QK
- * into that buffer may start), 10 scores in registers, 11 own row maxima known,
- * 12 running max of tile j-1 received, 13 the PV issuer saw the probabilities, 14 the PV
- * issuer saw O ready, 15 probabilities handed over by the softmax warp of the last row
- * quarter (event 2 is the first quarter's).  Reproduces the QK/PV overlap measurement of "Phase 2B
- * Aligned Numerical Prototype", Synchronization And Safety.  Same output as h3attn_attend. */
+ * happen are left untouched).  slot = the Q tile of the pair (0 or 1) the event belongs to;
+ * K-tile events use slot 0.  Events: 0 scores ready in the softmax warpgroup, 1 running max
+ * of tile j published to the correction, 2 probabilities handed to the PV issuer, 3 QK
+ * issued, 4 PV issued, 5 O rescaled (or left alone) by the correction warpgroup, 6 K tile
+ * landed, 7 probabilities computed (end of the MUFU turn), 8 PV issued and committed,
+ * 9 scores released (QK of tile j+1 may start), 10 scores in registers, 11 own row maxima
+ * known, 12 probability buffer free (PV of tile j-1 completed), 13 the PV issuer saw the
+ * probabilities, 14 the PV issuer saw O ready, 15 probabilities handed over by the softmax
+ * warp of the last row quarter (events 0-2, 7, 10-12 are the first quarter's).
+ * Reproduces the QK/PV overlap measurement of "Phase 2B Aligned Numerical Prototype",
+ * Synchronization And Safety.  Same output as h3attn_attend. */
 h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H,
                                         int D, float softmax_scale, const h3attn_bf16_out* out,
                                         int trace_block, uint64_t* trace_dev, void* stream);
