@@ -143,6 +143,39 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
                                      int D, int b, int h, int qt, int kt, int32_t* out_dev,
                                      void* stream);
 
+/* Device bytes h3attn_forward_host needs for these sizes and heads_per_group (two
+ * slots of staged Q, K, V and output plus a workspace for heads_per_group heads);
+ * 0 for invalid sizes or heads_per_group outside [1, H]. */
+size_t h3attn_forward_host_bytes(int B, int Tq, int Tkv, int H, int D, int heads_per_group);
+
+/* Forward pass (as h3attn_forward_ex) from HOST input views to a HOST output view, for
+ * callers whose activations are not resident on the device.  The heads are processed in
+ * groups of heads_per_group: group g is uploaded on an internal stream, computed on
+ * `stream`, and downloaded on a second internal stream, so the upload of group g+1 and
+ * the download of group g-1 overlap the kernels of group g.  Heads are independent
+ * problems (every statistic, scale and softmax is per (b, h)), so the result is bit for
+ * bit that of one h3attn_forward_ex call on all heads.
+ *   q, k, v, out: host views with the device views' rules (16-byte aligned data, strides
+ *     in elements, multiples of 8, channel stride 1); page-locked memory for the copies
+ *     to overlap.  The caller keeps them alive and unmodified until `stream` reaches the
+ *     end of the call (every copy of the call is ordered before that point).
+ *   dev_buf: device memory of h3attn_forward_host_bytes(...) bytes, 1024-byte aligned,
+ *     owned by the caller; holds the staging and the per-slot workspaces.
+ * Asynchronous on `stream`; creates its two copy streams and eight events per call and
+ * releases them before returning (the runtime frees them once their work is done).
+ * Device-side status: h3attn_forward_host_check_status.  The zero-copy layout of the
+ * north-star ("H3 Performance Roadmap", Phase 4 item 5: token-major in and out) applies
+ * to the host views the same way. */
+h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                  const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                  float softmax_scale, const h3attn_bf16_out* out, int heads_per_group,
+                                  void* dev_buf, size_t dev_bytes, void* stream);
+
+/* h3attn_check_status for the workspaces inside an h3attn_forward_host buffer: the
+ * first non-OK status of the slots the call used (each is read and cleared). */
+h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int Tkv, int H, int D,
+                                               int heads_per_group, void* stream);
+
 /* Failure-path test hook: h3attn_attend with every barrier wait bounded by
  * wait_limit_ns (1 ms to 2 s) and the correction warpgroup's "O ready" arrivals
  * withheld, so that the PV issuer's wait, and every wait behind it, has no

@@ -70,6 +70,12 @@ def lib() -> ctypes.CDLL:
         L.h3attn_debug_attend_trace.argtypes = [P, S] + [I] * 5 + [F, VP, I, P, P]
         L.h3attn_debug_attend_timeout.restype = I
         L.h3attn_debug_attend_timeout.argtypes = [P, S] + [I] * 5 + [F, VP, ctypes.c_uint64, P]
+        L.h3attn_forward_host_bytes.restype = S
+        L.h3attn_forward_host_bytes.argtypes = [I] * 6
+        L.h3attn_forward_host.restype = I
+        L.h3attn_forward_host.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, I, P, S, P]
+        L.h3attn_forward_host_check_status.restype = I
+        L.h3attn_forward_host_check_status.argtypes = [P] + [I] * 6 + [P]
         L.h3attn_status_string.restype = ctypes.c_char_p
         L.h3attn_status_string.argtypes = [I]
         L.h3attn_version.restype = I
@@ -164,6 +170,39 @@ def h3attn_forward(q, k, v, softmax_scale: float, out, ws, stream=None):
     vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
     _check(lib().h3attn_forward(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, T, H, D, softmax_scale,
                                 ctypes.byref(vo), wp, wb, _stream(stream)), "h3attn_forward")
+
+
+def h3attn_forward_host_bytes(B: int, Tq: int, Tkv: int, H: int, heads_per_group: int, D: int = HEAD_DIM) -> int:
+    return lib().h3attn_forward_host_bytes(B, Tq, Tkv, H, D, heads_per_group)
+
+
+def new_host_buffer(B: int, Tq: int, Tkv: int, H: int, heads_per_group: int, device="cuda"):
+    """Device buffer for h3attn_forward_host (1024-byte aligned: the allocation is rounded up and sliced)."""
+    import torch
+    n = h3attn_forward_host_bytes(B, Tq, Tkv, H, heads_per_group)
+    if n == 0:
+        raise H3AttnError(ERR_INVALID_ARG, "h3attn_forward_host_bytes")
+    raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    skip = (-raw.data_ptr()) % 1024
+    return raw[skip:skip + n]
+
+
+def h3attn_forward_host(q, k, v, softmax_scale: float, out, dev_buf, heads_per_group: int, stream=None):
+    """Forward pass from host q, k, v ([B, T, H, 128] BF16 CPU tensors, pinned for overlap) to a host
+    out view; dev_buf from new_host_buffer with the same sizes and heads_per_group."""
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(dev_buf)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib().h3attn_forward_host(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H, D,
+                                     softmax_scale, ctypes.byref(vo), heads_per_group, wp, wb, _stream(stream)),
+           "h3attn_forward_host")
+
+
+def h3attn_forward_host_check_status(dev_buf, B: int, Tq: int, Tkv: int, H: int, heads_per_group: int,
+                                     stream=None, D: int = HEAD_DIM) -> int:
+    return lib().h3attn_forward_host_check_status(dev_buf.data_ptr(), B, Tq, Tkv, H, D, heads_per_group,
+                                                  _stream(stream))
 
 
 STATIC_WS_BYTES = 64 << 20

@@ -99,6 +99,25 @@ def test_debug_export_rejects_out_of_range_tiles(L):
     assert f(ws, 1 << 40, 1, 256, 256, 2, 128, 0, 0, 0, 0, 0x3000004, None) == h3.ERR_ALIGNMENT
 
 
+def test_host_pipeline_sizes_and_argument_errors(L):
+    assert h3.h3attn_forward_host_bytes(1, 300, 300, 4, 0) == 0
+    assert h3.h3attn_forward_host_bytes(1, 300, 300, 4, 5) == 0
+    assert h3.h3attn_forward_host_bytes(1, 300, 300, 4, 2) == 2 * (h3.h3attn_forward_host_bytes(1, 300, 300, 2, 2) // 2)
+    good = _view(0x100000)
+    f = L.h3attn_forward_host
+    args = lambda q=good, out=None, g=2, buf=0x4000000, nbytes=1 << 40, D=128: f(
+        ctypes.byref(q) if q is not None else None, ctypes.byref(good), ctypes.byref(good), 1, 256, 256, 4, D, 0.088,
+        ctypes.byref(out if out is not None else _view(0x2000000)), g, buf, nbytes, None)
+    assert args(q=None) == h3.ERR_INVALID_ARG
+    assert args(g=0) == h3.ERR_INVALID_ARG
+    assert args(D=64) == h3.ERR_UNSUPPORTED
+    assert args(q=_view(0x100008)) == h3.ERR_ALIGNMENT
+    assert args(out=_view(0x2000000, st=4100)) == h3.ERR_ALIGNMENT
+    assert args(buf=0) == h3.ERR_WORKSPACE
+    assert args(buf=0x4000100) == h3.ERR_WORKSPACE
+    assert args(nbytes=1000) == h3.ERR_WORKSPACE
+
+
 def test_product_path_has_no_oracle_or_cpu_fallback():
     pkg = os.path.join(ROOT, "quantized_attention_video_b200")
     for dirpath, _, files in os.walk(pkg):
