@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(128) finalize_kernel(const double* __restrict_
   float* vp = vmax + bh * nchunk * kD + c;
   double s = 0.0;
   float m = 0.0f;
+  // the sum stays sequential in chunk order; unrolling lets the loads run ahead of it
+#pragma unroll 16
   for (int64_t ch = 0; ch < nchunk; ++ch) {
     s = __dadd_rn(s, kp[ch * kD]);
     m = fmaxf(m, vp[ch * kD]);
@@ -129,7 +131,19 @@ __device__ __forceinline__ float warp_max(float x) {
 
 // Thread (c16 = tid & 15, rq = tid >> 4) owns channels [8*c16, 8*c16+8) of the
 // 8 consecutive slab rows [8*rq, 8*rq+8).  Warp w covers slab rows [16w, 16w+16).
-__global__ void __launch_bounds__(256) quantize_kernel(
+// The Q and K row loads are issued before either is used and the V loads right
+// after the Q pass, so that a block keeps 64 KB in flight through its passes; the
+// raw BF16 words stay in registers until each tensor's pass unpacks them.
+__device__ __forceinline__ void load_rows(uint4 (&raw)[8], const uint16_t* p, int64_t st, int64_t t0, int rq,
+                                          int T) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int64_t t = t0 + 8 * rq + r;
+    raw[r] = t < T ? ldg16(p + t * st) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__global__ void __launch_bounds__(256, 2) quantize_kernel(
     const uint16_t* __restrict__ q, int64_t qsb, int64_t qst, int64_t qsh,
     const uint16_t* __restrict__ k, int64_t ksb, int64_t kst, int64_t ksh,
     const uint16_t* __restrict__ v, int64_t vsb, int64_t vst, int64_t vsh,
@@ -146,22 +160,22 @@ __global__ void __launch_bounds__(256) quantize_kernel(
   const int64_t t0 = (int64_t)blockIdx.x * kTile;
   const int64_t h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = b * H + h;
+  const bool has_q = t0 < Tq_pad, has_kv = t0 < Tkv_pad;
+
+  // padding rows (t >= T) load as zero words (BF16 +0)
+  uint4 rq8[8], rk8[8], rv8[8];
+  load_rows(rq8, q + b * qsb + h * qsh + c16 * 8, qst, t0, rq, has_q ? Tq : 0);
+  load_rows(rk8, k + b * ksb + h * ksh + c16 * 8, kst, t0, rq, has_kv ? Tkv : 0);
 
   // ---------------------------------------------------------------- Q ----
-  if (t0 < Tq_pad) {
-    float x[8][8];
+  if (has_q) {
     float amax = 0.0f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int64_t t = t0 + 8 * rq + r;
-      if (t < Tq) {
-        unpack8(ldg16(q + b * qsb + t * qst + h * qsh + c16 * 8), x[r]);
-      } else {
+      float x[8];
+      unpack8(rq8[r], x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[r][e] = 0.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[r][e]));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
     }
     amax = warp_max(amax);
     if (lane == 0) red[warp] = amax;
@@ -176,33 +190,35 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int64_t t = t0 + 8 * rq + r;
-      store_words(q8 + (bh * Tq_pad + t) * kD + c16 * 8, x[r], inv);
+      float x[8];
+      unpack8(rq8[r], x);
+      store_words(q8 + (bh * Tq_pad + t0 + 8 * rq + r) * kD + c16 * 8, x, inv);
     }
     __syncthreads();
   }
 
-  if (t0 >= Tkv_pad) return;
+  if (!has_kv) return;
+  load_rows(rv8, v + b * vsb + h * vsh + c16 * 8, vst, t0, rq, Tkv);
   // ---------------------------------------------------------------- K ----
   {
     float kmv[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) kmv[e] = km[bh * kD + c16 * 8 + e];
-    float x[8][8];
+    // smoothed values of valid rows; padding rows stay exactly 0
+    const auto smooth = [&](int r, float (&x)[8]) {
+      unpack8(rk8[r], x);
+      if (t0 + 8 * rq + r < Tkv) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], kmv[e]);
+      }
+    };
     float amax = 0.0f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int64_t t = t0 + 8 * rq + r;
-      if (t < Tkv) {
-        unpack8(ldg16(k + b * ksb + t * kst + h * ksh + c16 * 8), x[r]);
+      float x[8];
+      smooth(r, x);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], kmv[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[r][e] = 0.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[r][e]));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
     }
     amax = warp_max(amax);
     if (lane == 0) red[warp] = amax;
@@ -217,8 +233,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int64_t t = t0 + 8 * rq + r;
-      store_words(k8 + (bh * Tkv_pad + t) * kD + c16 * 8, x[r], inv);
+      float x[8];
+      smooth(r, x);
+      store_words(k8 + (bh * Tkv_pad + t0 + 8 * rq + r) * kD + c16 * 8, x, inv);
     }
   }
   // ---------------------------------------------------------------- V ----
@@ -229,22 +246,25 @@ __global__ void __launch_bounds__(256) quantize_kernel(
       const float a = vmax[bh * nchunk * kD + c16 * 8 + e];
       inv[e] = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
     }
-    uint8_t w[8][8];  // [channel e][row r]
+    // byte r of lo[e] / hi[e]: channel e of row r / r + 4 (E4M3)
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) lo[e] = hi[e] = 0u;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const int64_t t = t0 + 8 * rq + r;
       float x[8];
-      if (t < Tkv) {
-        unpack8(ldg16(v + b * vsb + t * vst + h * vsh + c16 * 8), x);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.0f;
-      }
+      unpack8(rv8[r], x);
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
         const uint32_t p = cvt_e4m3x2(__fmul_rn(x[e], inv[e]), __fmul_rn(x[e + 1], inv[e + 1]));
-        w[e][r] = (uint8_t)(p & 0xFF);
-        w[e + 1][r] = (uint8_t)(p >> 8);
+        const int sh = 8 * (r & 3);
+        if (r < 4) {
+          lo[e] |= (p & 0xFFu) << sh;
+          lo[e + 1] |= (p >> 8) << sh;
+        } else {
+          hi[e] |= (p & 0xFFu) << sh;
+          hi[e + 1] |= (p >> 8) << sh;
+        }
       }
     }
     // rows [8rq, 8rq+8) of channel c are bytes [8rq, 8rq+8) of smem row c; the
@@ -253,13 +273,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     for (int e = 0; e < 8; ++e) {
       const int c = c16 * 8 + e;
       const int chunk = (rq >> 1) ^ ((c >> 3) & 7);
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        lo |= (uint32_t)w[e][r] << (8 * r);
-        hi |= (uint32_t)w[e][r + 4] << (8 * r);
-      }
-      *reinterpret_cast<uint2*>(vt + c * kTile + chunk * 16 + (rq & 1) * 8) = make_uint2(lo, hi);
+      *reinterpret_cast<uint2*>(vt + c * kTile + chunk * 16 + (rq & 1) * 8) = make_uint2(lo[e], hi[e]);
     }
     __syncthreads();
 #pragma unroll
