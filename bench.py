@@ -32,6 +32,14 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 METRIC = "quantized attention effective TOPS and ms/call at T=37,810, H=32, D=128 (1xB200)"
+
+
+def metric_of(w) -> str:
+    """The headline metric string; other workloads name their own sizes."""
+    if w.name == DEFAULT_WORKLOAD:
+        return METRIC
+    return "quantized attention effective TOPS and ms/call at Tq=%s, Tkv=%s, B=%d, H=%d, D=%d (1xB200)" % (
+        format(w.Tq, ","), format(w.Tkv, ","), w.B, w.H, w.D)
 UNIT = "TOPS"
 DEFAULT_WORKLOAD = "h3_t37810_h32"
 KERNEL_SOURCES = ["quantized_attention_video_b200/csrc/attention.cu", "quantized_attention_video_b200/csrc/sm100_ptx.cuh"]
@@ -117,7 +125,7 @@ def run_reference(args, w):
         info = (threads, text)
     value = statistics.median(vals)
     ms = 4.0 * w.B * w.Tq * w.Tkv * w.H * w.D / (value * 1e12) * 1e3
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic",
             "config": config_of(w, 1),
@@ -172,13 +180,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def traffic_record():
+def traffic_record(w):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
+    taken on the current kernel source and this workload (else None)."""
     path = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path))
+    if rec.get("workload") != w.name:
+        return None
     h = hashlib.sha256()
     for src in KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, src), "rb").read())
@@ -322,7 +332,7 @@ def run_ours(args, w):
         peak = 2.0 * 1400.0
         peak_note = "of fallback: 2 x 1.4 PFLOP/s sustained bf16"
     achieved = ops / (attn_avg * 1e-3) / 1e12
-    tr = traffic_record()
+    tr = traffic_record(w)
     roofline = {"bound": "tensor", "kernel": "attn_sm100_kernel", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_note,
                 "algorithmic_ops_per_launch": ops,
@@ -342,7 +352,7 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if rank != 0:
         return
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+    line = {"metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic", "config": config_of(w, world),
             "clocks": clk, "gpu_launches": 4 * K, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu}

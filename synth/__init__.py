@@ -89,6 +89,8 @@ WORKLOADS = {
     "h3_t37810_h32": Workload("h3_t37810_h32", 1, 37810, 37810, 32, 128, "rmsnorm", 37810),
     "h3_packed_b2_t37810": Workload("h3_packed_b2_t37810", 2, 37810, 37810, 32, 128, "rmsnorm", 37811,
                                     packed=True),
+    # the pages' second required shape, "74K tokens" (the 243-frame workload), read as 74,000
+    "h3_t74000_h32": Workload("h3_t74000_h32", 1, 74000, 74000, 32, 128, "rmsnorm", 74000),
 }
 
 

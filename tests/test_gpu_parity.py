@@ -123,7 +123,7 @@ def run_forward(w, d):
 
 # ---------------------------------------------------------------- configs ----
 FULL = ["fixed_q128_kv192", "selfattn_h8_t4096"]
-SAMPLED = {"ragged_h16_t9453": 3, "h3_t37810_h32": 1, "h3_packed_b2_t37810": 0}
+SAMPLED = {"ragged_h16_t9453": 3, "h3_t37810_h32": 1, "h3_packed_b2_t37810": 0, "h3_t74000_h32": 0}
 
 
 @pytest.mark.parametrize("name", FULL + list(SAMPLED))
