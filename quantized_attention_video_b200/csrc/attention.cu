@@ -183,34 +183,48 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
 }
 
 
-// Scaled probabilities of the 128 keys of a row: q = 2^(s*f - mq) with
-// mq = m - log2(448), i.e. q = 448 * 2^(t - m); FP32 partial sums of q
-// into acc2 and the E4M3 words of q into w (4 keys per word).  kFmaExp2PairsOf8
-// key pairs in every eight take their exp2 from the FMA pipe (exp2_fma_pair),
-// the rest from MUFU.  The exp2 is volatile so that it stays after the MUFU
-// turn's wait; the FMA, add and conversion work around it fills the MUFU
-// latency.
-template <bool kMasked>
-__device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
-                                         uint64_t (&acc2)[4], uint32_t (&w)[32]) {
+// Softmax arithmetic of one row (128 keys, one per register), in two parts so that
+// only MUFU work needs the MUFU turn:
+//   pre_turn   in place, before the turn: u = s*f - mq (FP32 FMA; mq = m - log2(448),
+//              so 2^u = 448 * 2^(t - m)), and for kFmaExp2PairsOf8 of every 8 key
+//              pairs already q = 2^u by the FMA-pipe polynomial (exp2_fma_pair);
+//   probs128   in the turn: q = 2^u on MUFU for the other pairs, FP32 partial sums of q
+//              into acc2 and the E4M3 words of q into w (4 keys per word); with
+//              kMasked, keys >= valid give 0.  The sums and conversions of every pair
+//              fill the MUFU latency.  The MUFU exp2 is volatile so that it stays
+//              after the turn's wait.
+__device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1, float mq) {
   const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
   const uint64_t negm = f2_pack(-mq, -mq);
+#pragma unroll
+  for (int i = 0; i < 128; i += 2) {
+    const uint64_t u = f2_fma(f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1])), i < 64 ? ff0 : ff1, negm);
+    float q0, q1;
+    if (((i >> 1) & 7) < kFmaExp2PairsOf8)
+      exp2_fma_pair(u, q0, q1);
+    else
+      f2_unpack(u, q0, q1);
+    x[i] = __float_as_uint(q0);
+    x[i + 1] = __float_as_uint(q1);
+  }
+  // every value exists here: none of this work is left for the turn
+#pragma unroll
+  for (int i = 0; i < 128; ++i) asm volatile("" : "+r"(x[i]));
+}
+
+template <bool kMasked>
+__device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, uint64_t (&acc2)[4],
+                                         uint32_t (&w)[32]) {
 #pragma unroll
   for (int e = 0; e < 128; e += 4) {
     uint32_t half[2];
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int i = e + 2 * hp;
-      const uint64_t a = f2_pack(__uint_as_float(x[i]), __uint_as_float(x[i + 1]));
-      const uint64_t u = f2_fma(a, i < 64 ? ff0 : ff1, negm);
-      float q0, q1;
-      if (((i >> 1) & 7) < kFmaExp2PairsOf8) {
-        exp2_fma_pair(u, q0, q1);
-      } else {
-        float u0, u1;
-        f2_unpack(u, u0, u1);
-        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(u0));
-        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(u1));
+      float q0 = __uint_as_float(x[i]), q1 = __uint_as_float(x[i + 1]);
+      if (((i >> 1) & 7) >= kFmaExp2PairsOf8) {
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
       }
       if (kMasked) {
         if (i >= valid) q0 = 0.0f;
@@ -636,6 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
       const float mq = __fsub_rn(m_j, kLog2_448);
+      pre_turn(xs, f0, f1, mq);
       // MUFU turn: the exp2 passes alternate A(0) B(0) A(1) B(1) ... so that
       // each runs with the MUFU unit to itself while the other warpgroup does
       // the rest of its tile.
@@ -649,9 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (valid < kTile)
-        probs128<true>(xs, valid, f0, f1, mq, acc2, pw);
+        probs128<true>(xs, valid, acc2, pw);
       else
-        probs128<false>(xs, valid, f0, f1, mq, acc2, pw);
+        probs128<false>(xs, valid, acc2, pw);
       mbar_arrive(&sm.tok[x]);
       if (tr) trace(kEvProbs, x, j);
       if (j >= 1) {
