@@ -197,6 +197,22 @@ def traffic_record(w):
     return rec
 
 
+def max_over_ranks(dist, val: float, device) -> float:
+    """The slowest rank's value (all ranks take part; dist None = single process)."""
+    if dist is None:
+        return val
+    import torch
+    t = torch.tensor([val], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(ops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput of independent replicas (weak scaling): every rank does
+    ops_per_rank per step and the job is as slow as its slowest rank.  TOPS."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------- GPU arm ----
 def run_ours(args, w):
     import torch
@@ -267,18 +283,11 @@ def run_ours(args, w):
     if h3.h3attn_check_status(ws, stream) != h3.OK:
         raise RuntimeError("device status not OK after the timed steps")
 
-    def max_over_ranks(val):
-        if dist is None:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(dist, total_ms, dev)
     ms_step = total_ms / K
-    value = world * ops / (ms_step * 1e-3) / 1e12
-    attn_avg = max_over_ranks(statistics.mean(attn_ms))
-    quant_avg = max_over_ranks(statistics.mean(quant_ms))
+    value = job_rate(ops, world, ms_step)
+    attn_avg = max_over_ranks(dist, statistics.mean(attn_ms), dev)
+    quant_avg = max_over_ranks(dist, statistics.mean(quant_ms), dev)
 
     # ------------------------------------------------ end to end (host buffers)
     e2e = None
@@ -313,8 +322,8 @@ def run_ours(args, w):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke)
-        e2e = {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms, "steps": Ke,
+        e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ke, dev)
+        e2e = {"value": job_rate(ops, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms, "steps": Ke,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "pinned host Q/K/V -> h3attn_forward_host (upload, forward and download of head groups of %d "
                        "on overlapping streams) -> pinned host out" % g}
