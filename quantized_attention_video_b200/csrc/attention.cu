@@ -110,7 +110,8 @@ static_assert(sizeof(AttnSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
-  kSiteSoftS, kSiteSoftM, kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi, kSiteSoftTok
+  kSiteSoftS, kSiteSoftM /* unused: the running max no longer crosses warpgroups; kept so ids stay fixed */,
+  kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi, kSiteSoftTok
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
