@@ -305,3 +305,25 @@ def test_full_size_soak_is_deterministic_and_never_times_out():
     # no launch may stall: the slowest stays within 1.5x of the median
     times.sort()
     assert times[-1] < 1.5 * times[len(times) // 2], times
+
+
+def test_trace_export_gives_the_same_output_and_a_timeline():
+    """h3attn_debug_attend_trace runs the same kernel with a clock64 timeline in one CTA:
+    the output bytes equal h3attn_attend's, and the traced CTA's per-tile events are
+    ordered (scores ready -> probabilities computed -> handed over, tile after tile)."""
+    w = synth.WORKLOADS["selfattn_h8_t4096"]
+    x = synth.make_inputs(w)
+    d = upload(x, w)
+    ws, out, out4 = run_forward(w, d)
+    traced = torch.empty_like(out4)
+    ntq = -(-w.Tq // 128)
+    ctas = ((ntq + 1) // 2) * w.H * w.B
+    tr = h3.h3attn_debug_attend_trace(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, traced, ctas // 2)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    assert torch.equal(traced.view(torch.int16), out4.view(torch.int16))
+    nkv = -(-w.Tkv // 128)
+    for slot in (0, 1):
+        s_ready, probs, p_done = (tr[n][slot].numpy().astype(np.int64) for n in ("s_ready", "probs", "p_done"))
+        assert (s_ready > 0).all() and (probs > 0).all() and (p_done > 0).all()
+        assert (s_ready < probs).all() and (probs < p_done).all()
+        assert (np.diff(s_ready) > 0).all() and len(s_ready) == nkv
