@@ -327,3 +327,30 @@ def test_trace_export_gives_the_same_output_and_a_timeline():
         assert (s_ready > 0).all() and (probs > 0).all() and (p_done > 0).all()
         assert (s_ready < probs).all() and (probs < p_done).all()
         assert (np.diff(s_ready) > 0).all() and len(s_ready) == nkv
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """The forward pass (four launches, no host synchronisation) can be captured once into a
+    CUDA graph and replayed: every replay gives the bytes of a direct call."""
+    w = synth.WORKLOADS["fixed_q128_kv192"]
+    x = synth.make_inputs(w)
+    d = upload(x, w)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    direct = torch.empty(1, 128, 1, 128, dtype=torch.bfloat16, device="cuda")
+    h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, direct, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    out = torch.zeros_like(direct)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up on the capture stream
+        h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, out, ws)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, out, ws)
+    for _ in range(50):
+        out.zero_()
+        g.replay()
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(out.view(torch.int16), direct.view(torch.int16))
+    assert h3.h3attn_check_status(ws) == h3.OK
