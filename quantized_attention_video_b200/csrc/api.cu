@@ -28,14 +28,6 @@ h3attn_status check_sizes(int B, int Tq, int Tkv, int H, int D) {
   return H3ATTN_OK;
 }
 
-h3attn_status check_strides(const void* data, int64_t sb, int64_t st, int64_t sh) {
-  if (data == nullptr) return H3ATTN_ERR_INVALID_ARG;
-  if (sb < 0 || st < 0 || sh < 0) return H3ATTN_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(data) % 16 != 0) return H3ATTN_ERR_ALIGNMENT;
-  if (sb % 8 != 0 || st % 8 != 0 || sh % 8 != 0) return H3ATTN_ERR_ALIGNMENT;
-  return H3ATTN_OK;
-}
-
 h3attn_status check_view(const h3attn_bf16_view* v) {
   if (v == nullptr) return H3ATTN_ERR_INVALID_ARG;
   return check_strides(v->data, v->stride_b, v->stride_t, v->stride_h);

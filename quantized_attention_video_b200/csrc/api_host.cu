@@ -42,14 +42,6 @@ bool make_slot(int B, int Tq, int Tkv, int g, Slot* s) {
   return true;
 }
 
-h3attn_status check_host_view(const void* data, int64_t sb, int64_t st, int64_t sh) {
-  if (data == nullptr) return H3ATTN_ERR_INVALID_ARG;
-  if (sb < 0 || st < 0 || sh < 0) return H3ATTN_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(data) % 16 != 0) return H3ATTN_ERR_ALIGNMENT;
-  if (sb % 8 != 0 || st % 8 != 0 || sh % 8 != 0) return H3ATTN_ERR_ALIGNMENT;
-  return H3ATTN_OK;
-}
-
 // Heads [h0, h0 + gn) of a strided [B, T, H, D] host view <-> compact [B, T, gn, D]
 // device staging.  One 2D copy per batch item when the heads of a token are adjacent,
 // else one per (batch item, head).
@@ -93,11 +85,11 @@ h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_v
   if (need == 0) return D != kD ? H3ATTN_ERR_UNSUPPORTED : H3ATTN_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return H3ATTN_ERR_INVALID_ARG;
   for (const h3attn_bf16_view* hv : {q, k, v}) {
-    const h3attn_status st = check_host_view(hv->data, hv->stride_b, hv->stride_t, hv->stride_h);
+    const h3attn_status st = check_strides(hv->data, hv->stride_b, hv->stride_t, hv->stride_h);
     if (st != H3ATTN_OK) return st;
   }
   {
-    const h3attn_status st = check_host_view(out->data, out->stride_b, out->stride_t, out->stride_h);
+    const h3attn_status st = check_strides(out->data, out->stride_b, out->stride_t, out->stride_h);
     if (st != H3ATTN_OK) return st;
   }
   if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return H3ATTN_ERR_INVALID_ARG;

@@ -58,6 +58,16 @@ inline Layout make_layout(const Shape& s) {
   return L;
 }
 
+// A strided BF16 view's pointer and strides (elements): non-null, 16-byte aligned
+// data, non-negative strides that are multiples of 8 elements (16-byte vectors).
+inline h3attn_status check_strides(const void* data, int64_t sb, int64_t st, int64_t sh) {
+  if (data == nullptr) return H3ATTN_ERR_INVALID_ARG;
+  if (sb < 0 || st < 0 || sh < 0) return H3ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(data) % 16 != 0) return H3ATTN_ERR_ALIGNMENT;
+  if (sb % 8 != 0 || st % 8 != 0 || sh % 8 != 0) return H3ATTN_ERR_ALIGNMENT;
+  return H3ATTN_OK;
+}
+
 // Device-side status words at the start of the workspace.
 struct DevStatus {
   int code;    // h3attn_status of the first failure, 0 if none
