@@ -25,6 +25,9 @@
 namespace h3 {
 namespace {
 
+// Sequences of at most this many 128-token slabs take the one-launch preparation.
+constexpr int64_t kSmallSlabs = 4;
+
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -38,23 +41,37 @@ __device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// All three kernels take the same arguments.
+struct PrepParams {
+  const uint16_t* q;
+  int64_t qsb, qst, qsh;
+  const uint16_t* k;
+  int64_t ksb, kst, ksh;
+  const uint16_t* v;
+  int64_t vsb, vst, vsh;
+  int H, Tq, Tkv;
+  int64_t Tq_pad, Tkv_pad, nchunk, nunits;
+  double* ksum;  // [B, H, nchunk, 128] FP64 K chunk sums
+  float* vmax;   // [B, H, nchunk, 128] V chunk absmax; chunk row 0 ends as the channel absmax
+  float* km;
+  float* sv;
+  uint16_t* q8;
+  float* sq;
+  uint16_t* k8;
+  float* sk;
+  uint8_t* v8t;
+  DevStatus* status;
+};
+
 // ------------------------------------------------------------------ stats ----
-// Thread (unit, sub): unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice.
-__global__ void __launch_bounds__(256) stats_kernel(const uint16_t* __restrict__ k, int64_t ksb, int64_t kst,
-                                                    int64_t ksh, const uint16_t* __restrict__ v, int64_t vsb,
-                                                    int64_t vst, int64_t vsh, int H, int Tkv, int64_t nchunk,
-                                                    int64_t nunits, double* __restrict__ ksum,
-                                                    float* __restrict__ vmax) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t unit = g >> 4;
-  const int sub = (int)(g & 15);
-  if (unit >= nunits) return;
-  const int64_t chunk = unit % nchunk, bh = unit / nchunk;
-  const int64_t h = bh % H, b = bh / H;
+// One (unit, sub) pair: unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice.
+__device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, int sub) {
+  const int64_t chunk = unit % p.nchunk, bh = unit / p.nchunk;
+  const int64_t h = bh % p.H, b = bh / p.H;
   const int t0 = (int)(chunk * kChunk);
-  const int t1 = min(Tkv, t0 + kChunk);
-  const uint16_t* kp = k + b * ksb + h * ksh + sub * 8;
-  const uint16_t* vp = v + b * vsb + h * vsh + sub * 8;
+  const int t1 = min(p.Tkv, t0 + kChunk);
+  const uint16_t* kp = p.k + b * p.ksb + h * p.ksh + sub * 8;
+  const uint16_t* vp = p.v + b * p.vsb + h * p.vsh + sub * 8;
   double acc[8];
   float vm[8];
 #pragma unroll
@@ -62,47 +79,57 @@ __global__ void __launch_bounds__(256) stats_kernel(const uint16_t* __restrict__
 #pragma unroll 4
   for (int t = t0; t < t1; ++t) {
     float kf[8], vf[8];
-    unpack8(ldg16(kp + (int64_t)t * kst), kf);
-    unpack8(ldg16(vp + (int64_t)t * vst), vf);
+    unpack8(ldg16(kp + (int64_t)t * p.kst), kf);
+    unpack8(ldg16(vp + (int64_t)t * p.vst), vf);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       acc[e] = __dadd_rn(acc[e], (double)kf[e]);
       vm[e] = fmaxf(vm[e], fabsf(vf[e]));
     }
   }
-  double* ko = ksum + unit * kD + sub * 8;
-  float* vo = vmax + unit * kD + sub * 8;
+  double* ko = p.ksum + unit * kD + sub * 8;
+  float* vo = p.vmax + unit * kD + sub * 8;
 #pragma unroll
   for (int e = 0; e < 8; ++e) { ko[e] = acc[e]; vo[e] = vm[e]; }
 }
 
+// Thread (unit, sub) of the whole grid.
+__global__ void __launch_bounds__(256) stats_kernel(const PrepParams p) {
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if ((g >> 4) < p.nunits) stats_unit(p, g >> 4, (int)(g & 15));
+}
+
 // --------------------------------------------------------------- finalize ----
-// One block of 128 threads per (b, h); thread = channel.  After it runs, chunk
-// row 0 of the V-absmax scratch holds the channel absmax over all keys.  It
-// also clears the workspace status word, so each quantize call starts clean.
-__global__ void __launch_bounds__(128) finalize_kernel(const double* __restrict__ ksum, float* __restrict__ vmax,
-                                                       int64_t nchunk, int Tkv, float* __restrict__ km,
-                                                       float* __restrict__ sv, DevStatus* status) {
-  const int64_t bh = blockIdx.x;
-  const int c = threadIdx.x;
-  if (bh == 0 && c == 0) {
-    status->code = 0;
-    status->detail = 0;
-    status->block = 0;
-  }
-  const double* kp = ksum + bh * nchunk * kD + c;
-  float* vp = vmax + bh * nchunk * kD + c;
+// Channel c of (b, h): K mean = (sum of the chunk sums in chunk order) / Tkv, rounded
+// to FP32; V absmax over all keys (left in chunk row 0 of the V-absmax scratch) and the
+// V scale amax/448.
+__device__ __forceinline__ void finalize_channel(const PrepParams& p, int64_t bh, int c) {
+  const double* kp = p.ksum + bh * p.nchunk * kD + c;
+  float* vp = p.vmax + bh * p.nchunk * kD + c;
   double s = 0.0;
   float m = 0.0f;
   // the sum stays sequential in chunk order; unrolling lets the loads run ahead of it
 #pragma unroll 16
-  for (int64_t ch = 0; ch < nchunk; ++ch) {
+  for (int64_t ch = 0; ch < p.nchunk; ++ch) {
     s = __dadd_rn(s, kp[ch * kD]);
     m = fmaxf(m, vp[ch * kD]);
   }
-  km[bh * kD + c] = __double2float_rn(__ddiv_rn(s, (double)Tkv));
-  sv[bh * kD + c] = __fdiv_rn(m, 448.0f);
+  p.km[bh * kD + c] = __double2float_rn(__ddiv_rn(s, (double)p.Tkv));
+  p.sv[bh * kD + c] = __fdiv_rn(m, 448.0f);
   vp[0] = m;
+}
+
+// Clears the workspace status word, so each quantize call starts clean.
+__device__ __forceinline__ void clear_status(const PrepParams& p) {
+  p.status->code = 0;
+  p.status->detail = 0;
+  p.status->block = 0;
+}
+
+// One block of 128 threads per (b, h); thread = channel.
+__global__ void __launch_bounds__(128) finalize_kernel(const PrepParams p) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) clear_status(p);
+  finalize_channel(p, blockIdx.x, threadIdx.x);
 }
 
 // --------------------------------------------------------------- quantize ----
@@ -143,22 +170,27 @@ __device__ __forceinline__ void load_rows(uint4 (&raw)[8], const uint16_t* p, in
   }
 }
 
-__global__ void __launch_bounds__(256, 2) quantize_kernel(
-    const uint16_t* __restrict__ q, int64_t qsb, int64_t qst, int64_t qsh,
-    const uint16_t* __restrict__ k, int64_t ksb, int64_t kst, int64_t ksh,
-    const uint16_t* __restrict__ v, int64_t vsb, int64_t vst, int64_t vsh,
-    int H, int Tq, int Tkv, int64_t Tq_pad, int64_t Tkv_pad, int64_t nchunk,
-    const float* __restrict__ km, const float* __restrict__ vmax,
-    uint16_t* __restrict__ q8, float* __restrict__ sq, uint16_t* __restrict__ k8, float* __restrict__ sk,
-    uint8_t* __restrict__ v8t) {
-  __shared__ float red[8];
-  __shared__ float gmax[4];
-  __shared__ __align__(16) uint8_t vt[kD * kTile];  // [channel][token], 16-byte chunks XOR-swizzled
+// Slab `slab` (128 tokens) of (b, h).  red, gmax and vt are the block's shared scratch.
+__device__ __forceinline__ void quantize_slab(const PrepParams& p, int64_t slab, int64_t h, int64_t b, float* red,
+                                              float* gmax, uint8_t* vt) {
+  const uint16_t* __restrict__ q = p.q;
+  const uint16_t* __restrict__ k = p.k;
+  const uint16_t* __restrict__ v = p.v;
+  const int64_t qsb = p.qsb, qst = p.qst, qsh = p.qsh, ksb = p.ksb, kst = p.kst, ksh = p.ksh;
+  const int64_t vsb = p.vsb, vst = p.vst, vsh = p.vsh;
+  const int H = p.H, Tq = p.Tq, Tkv = p.Tkv;
+  const int64_t Tq_pad = p.Tq_pad, Tkv_pad = p.Tkv_pad, nchunk = p.nchunk;
+  const float* __restrict__ km = p.km;
+  const float* __restrict__ vmax = p.vmax;
+  uint16_t* __restrict__ q8 = p.q8;
+  float* __restrict__ sq = p.sq;
+  uint16_t* __restrict__ k8 = p.k8;
+  float* __restrict__ sk = p.sk;
+  uint8_t* __restrict__ v8t = p.v8t;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, rq = tid >> 4;
-  const int64_t t0 = (int64_t)blockIdx.x * kTile;
-  const int64_t h = blockIdx.y, b = blockIdx.z;
+  const int64_t t0 = slab * kTile;
   const int64_t bh = b * H + h;
   const bool has_q = t0 < Tq_pad, has_kv = t0 < Tkv_pad;
 
@@ -287,31 +319,69 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(
   }
 }
 
+
+// Slab blockIdx.x of (b = blockIdx.z, h = blockIdx.y).
+__global__ void __launch_bounds__(256, 2) quantize_kernel(const PrepParams p) {
+  __shared__ float red[8];
+  __shared__ float gmax[4];
+  __shared__ __align__(16) uint8_t vt[kD * kTile];  // [channel][token], 16-byte chunks XOR-swizzled
+  quantize_slab(p, blockIdx.x, blockIdx.y, blockIdx.z, red, gmax, vt);
+}
+
+// Short sequences: the whole preparation of (b, h) = blockIdx.x in one block and one
+// launch (statistics, their ordered reduction, then every slab), the same arithmetic
+// as the three-kernel path.  Every stage's global writes are read by other threads of
+// the block only after a block barrier.
+__global__ void __launch_bounds__(256, 1) prep_small_kernel(const PrepParams p) {
+  __shared__ float red[8];
+  __shared__ float gmax[4];
+  __shared__ __align__(16) uint8_t vt[kD * kTile];
+  const int64_t bh = blockIdx.x;
+  if (bh == 0 && threadIdx.x == 0) clear_status(p);
+  for (int64_t c = threadIdx.x >> 4; c < p.nchunk; c += blockDim.x >> 4)
+    stats_unit(p, bh * p.nchunk + c, (int)(threadIdx.x & 15));
+  __syncthreads();
+  if (threadIdx.x < kD) finalize_channel(p, bh, threadIdx.x);
+  __syncthreads();
+  const int64_t slabs = (p.Tq_pad > p.Tkv_pad ? p.Tq_pad : p.Tkv_pad) / kTile;
+  for (int64_t slab = 0; slab < slabs; ++slab) quantize_slab(p, slab, bh % p.H, bh / p.H, red, gmax, vt);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
                             const Shape& s, const Layout& L, char* ws, cudaStream_t st) {
-  auto* ksum = reinterpret_cast<double*>(ws + L.off[H3ATTN_WS_KSUM]);
-  auto* vmax = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_VMAX]);
-  auto* km = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_KM]);
-  auto* sv = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SV]);
-  const int64_t nunits = (int64_t)s.B * s.H * s.nchunk;
-  const int64_t threads = nunits * 16;
-  stats_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-      static_cast<const uint16_t*>(k.data), k.stride_b, k.stride_t, k.stride_h,
-      static_cast<const uint16_t*>(v.data), v.stride_b, v.stride_t, v.stride_h, s.H, s.Tkv, s.nchunk, nunits,
-      ksum, vmax);
-  finalize_kernel<<<(unsigned)(s.B * s.H), 128, 0, st>>>(ksum, vmax, s.nchunk, s.Tkv, km, sv,
-                                                        reinterpret_cast<DevStatus*>(ws + L.off[H3ATTN_WS_STATUS]));
+  PrepParams p;
+  p.q = static_cast<const uint16_t*>(q.data);
+  p.qsb = q.stride_b; p.qst = q.stride_t; p.qsh = q.stride_h;
+  p.k = static_cast<const uint16_t*>(k.data);
+  p.ksb = k.stride_b; p.kst = k.stride_t; p.ksh = k.stride_h;
+  p.v = static_cast<const uint16_t*>(v.data);
+  p.vsb = v.stride_b; p.vst = v.stride_t; p.vsh = v.stride_h;
+  p.H = s.H; p.Tq = s.Tq; p.Tkv = s.Tkv;
+  p.Tq_pad = s.Tq_pad; p.Tkv_pad = s.Tkv_pad; p.nchunk = s.nchunk;
+  p.nunits = (int64_t)s.B * s.H * s.nchunk;
+  p.ksum = reinterpret_cast<double*>(ws + L.off[H3ATTN_WS_KSUM]);
+  p.vmax = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_VMAX]);
+  p.km = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_KM]);
+  p.sv = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SV]);
+  p.q8 = reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_Q8]);
+  p.sq = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SQ]);
+  p.k8 = reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_K8]);
+  p.sk = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SK]);
+  p.v8t = reinterpret_cast<uint8_t*>(ws + L.off[H3ATTN_WS_V8T]);
+  p.status = reinterpret_cast<DevStatus*>(ws + L.off[H3ATTN_WS_STATUS]);
   const int64_t slabs = (s.Tq_pad > s.Tkv_pad ? s.Tq_pad : s.Tkv_pad) / kTile;
+  if (slabs <= kSmallSlabs) {
+    // few tokens per head: one launch, one block per (b, h)
+    prep_small_kernel<<<(unsigned)((int64_t)s.B * s.H), 256, 0, st>>>(p);
+    return cudaGetLastError();
+  }
+  const int64_t threads = p.nunits * 16;
+  stats_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p);
+  finalize_kernel<<<(unsigned)(s.B * s.H), 128, 0, st>>>(p);
   dim3 grid((unsigned)slabs, (unsigned)s.H, (unsigned)s.B);
-  quantize_kernel<<<grid, 256, 0, st>>>(
-      static_cast<const uint16_t*>(q.data), q.stride_b, q.stride_t, q.stride_h,
-      static_cast<const uint16_t*>(k.data), k.stride_b, k.stride_t, k.stride_h,
-      static_cast<const uint16_t*>(v.data), v.stride_b, v.stride_t, v.stride_h, s.H, s.Tq, s.Tkv, s.Tq_pad,
-      s.Tkv_pad, s.nchunk, km, vmax, reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_Q8]),
-      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SQ]), reinterpret_cast<uint16_t*>(ws + L.off[H3ATTN_WS_K8]),
-      reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SK]), reinterpret_cast<uint8_t*>(ws + L.off[H3ATTN_WS_V8T]));
+  quantize_kernel<<<grid, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
