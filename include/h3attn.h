@@ -23,10 +23,14 @@
  *   out         = bf16((RO * (1/d)) * (sv/448))
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *     never allocates, never frees and never synchronises except in
- *     h3attn_check_status.  It keeps no state between calls other than a
- *     per-device cache of kernel attributes.
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except the
+ *     host views of h3attn_forward_host.  The library never allocates or frees
+ *     device memory and never synchronises except in h3attn_check_status (and
+ *     h3attn_forward_host_check_status); h3attn_forward_host creates two copy
+ *     streams and eight events per call and releases them before it returns, and
+ *     h3attn_forward_static uses its own static device array.  Other than that
+ *     array, the library keeps no state between calls beyond per-device caches of
+ *     kernel attributes and the array's address.
  *   - Element strides are in BF16 elements; the channel (d) stride is 1.
  *     Base pointers must be 16-byte aligned and strides multiples of 8
  *     elements (16-byte vector loads); the workspace must be 256-byte aligned.
@@ -105,8 +109,10 @@ h3attn_status h3attn_workspace_layout(int B, int Tq, int Tkv, int H, int D,
 /* K smoothing, Q/K INT8 and V FP8 quantization ("H3 Performance Roadmap", the
  * Sage2 decomposition: K smoothing, Q/K INT8 quantization, V transpose and FP8
  * quantization).  Reads q (Tq tokens) and k, v (Tkv tokens); writes every
- * field of the workspace except the status word.  Three kernels:
- * per-chunk statistics, their ordered reduction, one quantize pass. */
+ * field of the workspace and clears its status word.  Three kernels (per-chunk
+ * statistics, their ordered reduction, one quantize pass), or one kernel doing
+ * all three per (b, h) when max(Tq, Tkv) is at most 512 tokens; both give the
+ * same words. */
 h3attn_status h3attn_quantize_qkv(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
                                   const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
                                   void* ws, size_t ws_bytes, void* stream);
@@ -138,7 +144,11 @@ h3attn_status h3attn_check_status(void* ws, void* stream);
 
 /* Parity export: the exact INT32 QK^T tile of (b, h, Q tile qt, key tile kt) as
  * computed by the same tensor-core path the attention kernel uses, written as
- * 128 x 128 row-major int32 to the device buffer out_dev. */
+ * 128 x 128 row-major int32 to the device buffer out_dev (caller-owned, 16-byte
+ * aligned; rows or keys past Tq/Tkv hold the products of the zero padding).  ws must
+ * hold a quantize pass of the same sizes.  H3ATTN_ERR_INVALID_ARG for indices out of
+ * range or a null out_dev, H3ATTN_ERR_ALIGNMENT for a misaligned one.  The INT32
+ * score checkpoint of "Phase 2B Aligned Numerical Prototype", Exactness. */
 h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int Tq, int Tkv, int H,
                                      int D, int b, int h, int qt, int kt, int32_t* out_dev,
                                      void* stream);
