@@ -3,9 +3,14 @@
 // FP8 quantization; Phase 4 item 2: keep the per-warp INT8 Q/K and FP8 V policy).
 //
 //   stats_kernel    : one pass over K and V. Per (b, h, 64-token chunk, channel):
-//                     FP64 sum of K in token order, FP32 absmax of V.
+//                     FP64 sum of K in token order, FP32 absmax of V.  One block
+//                     per 128-token slab; the slab is staged in shared memory with
+//                     every load in flight before the in-order sums start.
 //   finalize_kernel : per (b, h, channel): K mean = (sum of chunk sums in chunk
 //                     order) / Tkv, rounded to FP32; V absmax and scale amax/448.
+//                     The chunk sums pass through shared memory in 256-chunk
+//                     passes, so that one warp's in-order sum never waits on a
+//                     global load.
 //   quantize_kernel : one pass over Q, K, V in 128-token slabs. INT8 Q per
 //                     32-token group, INT8 (K - mean) per 64-token group, FP8 E4M3
 //                     V per channel written transposed (channel-major), zero
@@ -18,6 +23,8 @@
 // All loads are 16-byte vectors of 8 BF16 channels; 16 threads cover one
 // 128-channel row, so a warp reads two contiguous 256-byte rows per load.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "h3attn_internal.h"
 #include "sm100_ptx.cuh"
@@ -50,7 +57,7 @@ struct PrepParams {
   const uint16_t* v;
   int64_t vsb, vst, vsh;
   int H, Tq, Tkv;
-  int64_t Tq_pad, Tkv_pad, nchunk, nunits;
+  int64_t Tq_pad, Tkv_pad, nchunk;
   double* ksum;  // [B, H, nchunk, 128] FP64 K chunk sums
   float* vmax;   // [B, H, nchunk, 128] V chunk absmax; chunk row 0 ends as the channel absmax
   float* km;
@@ -93,10 +100,71 @@ __device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, in
   for (int e = 0; e < 8; ++e) { ko[e] = acc[e]; vo[e] = vm[e]; }
 }
 
-// Thread (unit, sub) of the whole grid.
-__global__ void __launch_bounds__(256) stats_kernel(const PrepParams p) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if ((g >> 4) < p.nunits) stats_unit(p, g >> 4, (int)(g & 15));
+// Slab blockIdx.x (128 tokens = chunks 2x, 2x + 1) of (b = blockIdx.z, h = blockIdx.y).
+// Thread (c16 = tid & 15, r0 = tid >> 4) loads channels [8*c16, 8*c16+8) of slab rows
+// r0 + 16 i (i < 8; rows of chunk i / 4): sixteen 16-byte loads in flight per thread.
+// K goes to shared memory, where thread (chunk, channel) then adds its chunk's tokens
+// in token order; the V absmax is reduced from the registers (a max is exact in any
+// order).  The same sums and maxima as stats_unit.
+constexpr int kStatsThreads = 256;
+
+__global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p) {
+  __shared__ __align__(16) uint16_t ks[kTile * kD];                 // [row][channel] BF16
+  __shared__ float vred[kStatsThreads / 32][kTile / kChunk][kD];  // [warp][chunk][channel]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c16 = tid & 15, r0 = tid >> 4;
+  const int64_t slab = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = b * p.H + h, t0 = slab * kTile;
+  const uint16_t* kp = p.k + b * p.ksb + h * p.ksh + c16 * 8;
+  const uint16_t* vp = p.v + b * p.vsb + h * p.vsh + c16 * 8;
+  uint4 kr[8], vr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + r0 + 16 * i;
+    const bool in = t < p.Tkv;
+    kr[i] = in ? ldg16(kp + t * p.kst) : make_uint4(0u, 0u, 0u, 0u);
+    vr[i] = in ? ldg16(vp + t * p.vst) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(ks + (r0 + 16 * i) * kD + c16 * 8) = kr[i];
+  float vm[2][8];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vm[c][e] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float x[8];
+    unpack8(vr[i], x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vm[i >> 2][e] = fmaxf(vm[i >> 2][e], fabsf(x[e]));
+  }
+  // lanes l and l ^ 16 hold the same channels (slab rows 2w and 2w + 1 of each 16)
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vm[c][e] = fmaxf(vm[c][e], __shfl_xor_sync(0xFFFFFFFFu, vm[c][e], 16));
+  if (lane < 16) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) vred[warp][c][c16 * 8 + e] = vm[c][e];
+  }
+  __syncthreads();
+  const int ck = tid >> 7, ch = tid & (kD - 1);
+  const int64_t chunk = slab * (kTile / kChunk) + ck;
+  if (chunk >= p.nchunk) return;
+  const int n = (int)min((int64_t)kChunk, p.Tkv - chunk * kChunk);
+  const uint16_t* col = ks + ck * kChunk * kD + ch;
+  double acc = 0.0;
+#pragma unroll 16
+  for (int r = 0; r < n; ++r) acc = __dadd_rn(acc, (double)__uint_as_float((uint32_t)col[r * kD] << 16));
+  float m = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kStatsThreads / 32; ++w) m = fmaxf(m, vred[w][ck][ch]);
+  const int64_t unit = bh * p.nchunk + chunk;
+  p.ksum[unit * kD + ch] = acc;
+  p.vmax[unit * kD + ch] = m;
 }
 
 // --------------------------------------------------------------- finalize ----
@@ -126,10 +194,70 @@ __device__ __forceinline__ void clear_status(const PrepParams& p) {
   p.status->block = 0;
 }
 
-// One block of 128 threads per (b, h); thread = channel.
-__global__ void __launch_bounds__(128) finalize_kernel(const PrepParams p) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) clear_status(p);
-  finalize_channel(p, blockIdx.x, threadIdx.x);
+// Block (b*H + h = blockIdx.x, channels [32*blockIdx.y, 32*blockIdx.y + 32)); lane =
+// channel.  Pass q stages the chunk sums of chunks [256q, 256q + 256) in shared memory
+// (warp w loads 16 chunk rows, all in flight); warp 0 adds them in chunk order while
+// every warp's loads of pass q + 1 are in flight.  The same sum, mean, absmax and
+// scale as finalize_channel.
+constexpr int kFinThreads = 512;
+constexpr int kFinRowsPerWarp = 16;
+constexpr int kFinRows = kFinThreads / 32 * kFinRowsPerWarp;
+constexpr size_t kFinSmemBytes = 2 * (size_t)kFinRows * 32 * sizeof(double);
+
+__global__ void __launch_bounds__(kFinThreads) finalize_kernel(const PrepParams p) {
+  extern __shared__ __align__(16) double fin[];  // [2][kFinRows][32]
+  __shared__ float vred[kFinThreads / 32][32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t bh = blockIdx.x;
+  const int c = blockIdx.y * 32 + lane;
+  if (bh == 0 && blockIdx.y == 0 && tid == 0) clear_status(p);
+  const double* kp = p.ksum + bh * p.nchunk * kD + c;
+  float* vp = p.vmax + bh * p.nchunk * kD + c;
+  const int64_t npass = (p.nchunk + kFinRows - 1) / kFinRows;
+  double kr[kFinRowsPerWarp];
+  float vr[kFinRowsPerWarp];
+  float m = 0.0f;
+  const auto load = [&](int64_t q) {
+#pragma unroll
+    for (int i = 0; i < kFinRowsPerWarp; ++i) {
+      const int64_t ch = q * kFinRows + warp * kFinRowsPerWarp + i;
+      const bool in = ch < p.nchunk;
+      kr[i] = in ? kp[ch * kD] : 0.0;
+      vr[i] = in ? vp[ch * kD] : 0.0f;
+    }
+  };
+  const auto store = [&](int64_t q) {
+    double* dst = fin + ((q & 1) * kFinRows + warp * kFinRowsPerWarp) * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < kFinRowsPerWarp; ++i) {
+      dst[i * 32] = kr[i];
+      m = fmaxf(m, vr[i]);
+    }
+  };
+  load(0);
+  store(0);
+  __syncthreads();
+  double s = 0.0;
+  for (int64_t q = 0; q < npass; ++q) {
+    if (q + 1 < npass) load(q + 1);
+    if (warp == 0) {
+      const int n = (int)min((int64_t)kFinRows, p.nchunk - q * kFinRows);
+      const double* row = fin + (q & 1) * kFinRows * 32 + lane;
+#pragma unroll 16
+      for (int r = 0; r < n; ++r) s = __dadd_rn(s, row[r * 32]);
+    }
+    // buffer (q + 1) & 1 was last read by warp 0 in pass q - 1, before the barrier
+    if (q + 1 < npass) store(q + 1);
+    __syncthreads();
+  }
+  vred[warp][lane] = m;
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int w = 1; w < kFinThreads / 32; ++w) m = fmaxf(m, vred[w][lane]);
+  p.km[bh * kD + c] = __double2float_rn(__ddiv_rn(s, (double)p.Tkv));
+  p.sv[bh * kD + c] = __fdiv_rn(m, 448.0f);
+  vp[0] = m;
 }
 
 // --------------------------------------------------------------- quantize ----
@@ -347,6 +475,21 @@ __global__ void __launch_bounds__(256, 1) prep_small_kernel(const PrepParams p) 
   for (int64_t slab = 0; slab < slabs; ++slab) quantize_slab(p, slab, bh % p.H, bh / p.H, red, gmax, vt);
 }
 
+// The finalize kernel's shared memory is above the default 48 KB limit (set once per device).
+cudaError_t ensure_prep_attrs() {
+  static int done_mask = 0;  // one bit per device ordinal < 32
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 32 && (done_mask >> dev) & 1) return cudaSuccess;
+  e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinSmemBytes);
+  if (e != cudaSuccess) return e;
+  if (dev < 32) done_mask |= 1 << dev;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
@@ -360,7 +503,6 @@ cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k
   p.vsb = v.stride_b; p.vst = v.stride_t; p.vsh = v.stride_h;
   p.H = s.H; p.Tq = s.Tq; p.Tkv = s.Tkv;
   p.Tq_pad = s.Tq_pad; p.Tkv_pad = s.Tkv_pad; p.nchunk = s.nchunk;
-  p.nunits = (int64_t)s.B * s.H * s.nchunk;
   p.ksum = reinterpret_cast<double*>(ws + L.off[H3ATTN_WS_KSUM]);
   p.vmax = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_VMAX]);
   p.km = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_KM]);
@@ -377,9 +519,10 @@ cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k
     prep_small_kernel<<<(unsigned)((int64_t)s.B * s.H), 256, 0, st>>>(p);
     return cudaGetLastError();
   }
-  const int64_t threads = p.nunits * 16;
-  stats_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p);
-  finalize_kernel<<<(unsigned)(s.B * s.H), 128, 0, st>>>(p);
+  const cudaError_t e = ensure_prep_attrs();
+  if (e != cudaSuccess) return e;
+  stats_kernel<<<dim3((unsigned)(s.Tkv_pad / kTile), (unsigned)s.H, (unsigned)s.B), kStatsThreads, 0, st>>>(p);
+  finalize_kernel<<<dim3((unsigned)(s.B * s.H), kD / 32), kFinThreads, kFinSmemBytes, st>>>(p);
   dim3 grid((unsigned)slabs, (unsigned)s.H, (unsigned)s.B);
   quantize_kernel<<<grid, 256, 0, st>>>(p);
   return cudaGetLastError();
