@@ -66,6 +66,7 @@ def lib():
         L.orc_scores.argtypes = [_P, _P] + [_I] * 5 + [_I] * 6 + [_P]
         L.orc_attend_rows.argtypes = [_P] * 6 + [_I] * 7 + [_F, _I, _I, _P, _P, _P, _P]
         L.orc_row_trace.argtypes = [_P] * 6 + [_I] * 7 + [_F, _I, _I, _I, _I] + [_P] * 9
+        L.orc_qk_norm_rope.argtypes = [_P, _I64, _I64, _I64, _I, _I, _I, _I, _P, _F, _P, _P, _P]
         _lib = L
     return _lib
 
@@ -130,6 +131,32 @@ def quantize(q, k, v, gq: int = GQ, gk: int = GK) -> dict:
         raise ValueError("orc_quantize rejected its arguments")
     r.update(B=B, Tq=Tq, Tkv=Tkv, H=H, D=D, gq=gq, gk=gk)
     return r
+
+
+def qk_norm_rope(x, gamma, eps: float, cos, sin) -> np.ndarray:
+    """Per-head RMSNorm + interleaved-pair RoPE of a BF16 [B,T,H,D] view (oracle.cpp,
+    orc_qk_norm_rope, for the exact steps).  gamma [D], cos/sin [T, D/2] FP32.
+    Returns a dense [B,T,H,D] uint16 (BF16 bits) array."""
+    B, T, H, D = x.shape
+    gamma = np.ascontiguousarray(gamma, dtype=np.float32)
+    cos = np.ascontiguousarray(cos, dtype=np.float32)
+    sin = np.ascontiguousarray(sin, dtype=np.float32)
+    assert gamma.shape == (D,) and cos.shape == (T, D // 2) and sin.shape == (T, D // 2)
+    out = np.empty((B, T, H, D), np.uint16)
+    xa = _view_args(x)
+    rc = lib().orc_qk_norm_rope(xa[0], *xa[1:], B, T, H, D, gamma.ctypes.data, eps, cos.ctypes.data,
+                                sin.ctypes.data, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("orc_qk_norm_rope rejected its arguments")
+    return out
+
+
+def quantize_norm_rope(q, k, v, nr: dict, gq: int = GQ, gk: int = GK) -> dict:
+    """The preparation with Q/K RMSNorm + RoPE: qk_norm_rope on Q and on K, then quantize.
+    nr holds gamma_q, gamma_k, eps, cos_q, sin_q, cos_k, sin_k."""
+    qn = qk_norm_rope(q, nr["gamma_q"], nr["eps"], nr["cos_q"], nr["sin_q"])
+    kn = qk_norm_rope(k, nr["gamma_k"], nr["eps"], nr["cos_k"], nr["sin_k"])
+    return quantize(qn, kn, v, gq, gk)
 
 
 def _qz_args(z):

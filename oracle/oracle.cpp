@@ -32,6 +32,10 @@
 //     p = exp2(t - m) in FP32, stored as e4m3(448 * p); d sums the FP32 p.
 //   * RO <- RO*alpha + sum_j dec(p8_j)*dec(v8_jc), FP32, ascending j.
 //   * out = bf16((RO * (1/d)) * (sv/448)).
+//   * Optional Q/K RMSNorm + RoPE before quantization ("H3 Performance Roadmap",
+//     Component 2 execution order item 1 and the strided-NHD paragraph: Q/K
+//     normalization and RoPE applied where the attention consumes Q and K), see
+//     orc_qk_norm_rope: the quantization then reads its BF16 result.
 // Compiled with -ffp-contract=off so that no multiply-add is fused.
 #include <cmath>
 #include <cstdint>
@@ -228,6 +232,64 @@ int orc_quantize(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 for (int t = 0; t < Tkv; ++t) {
                     float x = bf16_decode(v[b * v_sb + t * v_st + h * v_sh + d]);
                     v8[(bh * Tkv + t) * D + d] = amax > 0.0f ? e4m3_encode(x * inv) : 0;
+                }
+            }
+        }
+    return 0;
+}
+
+// ------------------------------------------------------ Q/K norm + RoPE ----
+// Per-head RMSNorm over the D channels of each (b, t, h) row followed by the
+// rotary embedding of channel pairs (2i, 2i+1), the Q/K preparation that the
+// pages' H3 block runs before attention ("Norm and RoPE" in the representative
+// block table; fused into the attention's input path in Component 2, item 1).
+// The pages fix neither formula; the reading taken, step by step:
+//   ss  = sum of x_c^2 in FP32 (the precision RMSNorm layers usually accumulate
+//         in): the D/8 slices of 8 channels are each summed in channel order,
+//         then the slice sums are added pairwise, halving the count each time:
+//         slice s += slice s + w for s < w, w = D/16, ..., 2, 1 (for D = 128:
+//         s + 8, then s + 4, s + 2, s + 1); every product and sum is rounded
+//         separately;
+//   ms  = ss / D;  r = 1 / sqrt(ms + eps)   (FP32, each step rounded);
+//   n_c = bf16(x_c * r);  z_c = bf16(n_c * gamma_c)   (the norm output, BF16);
+//   out_2i   = bf16(z_2i * cos_i - z_2i+1 * sin_i)   (FP32, each product and the
+//   out_2i+1 = bf16(z_2i+1 * cos_i + z_2i * sin_i)    sum rounded; no FMA).
+// x is [B, T, H, D] BF16 with element strides (sb, st, sh); cos, sin are
+// [T, D/2] FP32 (row t = token t); out is dense [B, T, H, D] BF16.
+int orc_qk_norm_rope(const uint16_t* x, int64_t sb, int64_t st, int64_t sh, int B, int T, int H, int D,
+                     const float* gamma, float eps, const float* cosv, const float* sinv, uint16_t* out) {
+    if (B < 1 || T < 1 || H < 1 || D < 16 || D % 16 != 0 || !(eps > 0.0f)) return -1;
+    const int nslice = D / 8;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            std::vector<float> part(nslice);
+            std::vector<float> z(D);
+            for (int h = 0; h < H; ++h) {
+                const uint16_t* xr = x + b * sb + t * st + h * sh;
+                for (int s = 0; s < nslice; ++s) {
+                    float acc = 0.0f;
+                    for (int c = 8 * s; c < 8 * s + 8; ++c) {
+                        const float xc = bf16_decode(xr[c]);
+                        acc += xc * xc;
+                    }
+                    part[s] = acc;
+                }
+                for (int w = nslice / 2; w >= 1; w /= 2)
+                    for (int s = 0; s < w; ++s) part[s] += part[s + w];
+                const float ms = part[0] / (float)D;
+                const float den = std::sqrt(ms + eps);
+                const float r = 1.0f / den;
+                for (int c = 0; c < D; ++c) {
+                    const float n = bf16_decode(bf16_encode(bf16_decode(xr[c]) * r));
+                    z[c] = bf16_decode(bf16_encode(n * gamma[c]));
+                }
+                uint16_t* o = out + (((int64_t)b * T + t) * H + h) * D;
+                for (int i = 0; i < D / 2; ++i) {
+                    const float cs = cosv[(int64_t)t * (D / 2) + i], sn = sinv[(int64_t)t * (D / 2) + i];
+                    const float a = z[2 * i], bb = z[2 * i + 1];
+                    o[2 * i] = bf16_encode(a * cs - bb * sn);
+                    o[2 * i + 1] = bf16_encode(bb * cs + a * sn);
                 }
             }
         }

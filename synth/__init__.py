@@ -18,6 +18,14 @@ shapes of the H3 video-diffusion attention described on the pages:
   [2, T, 3, H, D] QKV buffer, output into [2, T, H*D].
 
 N(mu, v) names a normal with variance v.
+
+Workloads with ``norm_rope`` set feed raw projection-like Q/K (N(0,1)) through the
+Q/K RMSNorm + RoPE preparation: per-channel weights gamma_q, gamma_k ~ N(1, 0.1),
+eps = 1e-6, and rotary tables from ``rope_tables``: video tokens laid out in
+raster order on frames of 24 x 42 latent tokens, the 64 channel pairs split
+8 / 28 / 28 between the time, height and width positions, pair k of an axis with
+n pairs turning at theta^(-k/n) radians per position (theta = 256); the last 100
+tokens (the text) are left unrotated (cos 1, sin 0).
 """
 from __future__ import annotations
 
@@ -33,7 +41,13 @@ _SO = os.path.join(_HERE, "libsynth.so")
 _SRC = os.path.join(_HERE, "gen.c")
 
 NORMAL, OFFSET, RMSNORM = 0, 1, 2
-STREAM_Q, STREAM_K, STREAM_V, STREAM_GAMMA_Q, STREAM_GAMMA_K, STREAM_OFFSET_K = range(6)
+STREAM_Q, STREAM_K, STREAM_V, STREAM_GAMMA_Q, STREAM_GAMMA_K, STREAM_OFFSET_K, STREAM_NR_GAMMA_Q, STREAM_NR_GAMMA_K = \
+    range(8)
+ROPE_THETA = 256.0
+ROPE_PAIRS = (8, 28, 28)  # time, height, width (64 channel pairs)
+ROPE_FRAME = (24, 42)     # latent tokens per frame: height x width, raster order
+ROPE_TEXT = 100           # trailing tokens left unrotated
+NORM_EPS = 1e-6
 
 
 def build(force: bool = False) -> str:
@@ -71,6 +85,7 @@ class Workload:
     recipe: str          # "normal", "k_offset" or "rmsnorm"
     seed: int
     packed: bool = False  # Q/K/V read from one [B,T,3,H,D] buffer, out [B,T,H*D]
+    norm_rope: bool = False  # Q/K pass through the RMSNorm + RoPE preparation
 
     @property
     def scale(self) -> float:
@@ -91,7 +106,36 @@ WORKLOADS = {
                                     packed=True),
     # the pages' second required shape, "74K tokens" (the 243-frame workload), read as 74,000
     "h3_t74000_h32": Workload("h3_t74000_h32", 1, 74000, 74000, 32, 128, "rmsnorm", 74000),
+    # raw Q/K through the Q/K RMSNorm + RoPE preparation
+    "nr_h4_t1100": Workload("nr_h4_t1100", 1, 1100, 1100, 4, 128, "normal", 1100, norm_rope=True),
+    "h3_t37810_h32_nr": Workload("h3_t37810_h32_nr", 1, 37810, 37810, 32, 128, "normal", 37812,
+                                 norm_rope=True),
 }
+
+
+def rope_tables(T: int, n_text: int = ROPE_TEXT, frame=ROPE_FRAME, pairs=ROPE_PAIRS, theta: float = ROPE_THETA):
+    """Rotary tables cos, sin [T, 64] float32 of the layout described in the module docstring."""
+    assert sum(pairs) == 64
+    n_vid = max(0, T - n_text)
+    v = np.arange(n_vid)
+    per_frame = frame[0] * frame[1]
+    pos = (v // per_frame, (v % per_frame) // frame[1], v % frame[1])
+    ang = np.zeros((T, 64), dtype=np.float64)
+    col = 0
+    for axis, n in enumerate(pairs):
+        freq = theta ** (-np.arange(n, dtype=np.float64) / n)
+        ang[:n_vid, col:col + n] = pos[axis][:, None].astype(np.float64) * freq[None, :]
+        col += n
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def norm_rope_params(w: "Workload") -> dict:
+    """Host (numpy) parameters of the Q/K RMSNorm + RoPE of a norm_rope workload."""
+    cq, sq = rope_tables(w.Tq)
+    ck, sk = (cq, sq) if w.Tkv == w.Tq else rope_tables(w.Tkv)
+    return dict(gamma_q=normal_f32(w.D, w.seed, STREAM_NR_GAMMA_Q, 1.0, float(np.sqrt(0.1))),
+                gamma_k=normal_f32(w.D, w.seed, STREAM_NR_GAMMA_K, 1.0, float(np.sqrt(0.1))),
+                eps=NORM_EPS, cos_q=cq, sin_q=sq, cos_k=ck, sin_k=sk)
 
 
 def normal_f32(n: int, seed: int, stream: int, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
