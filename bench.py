@@ -38,8 +38,8 @@ def metric_of(w) -> str:
     """The headline metric string; other workloads name their own sizes."""
     if w.name == DEFAULT_WORKLOAD:
         return METRIC
-    return "quantized attention effective TOPS and ms/call at Tq=%s, Tkv=%s, B=%d, H=%d, D=%d (1xB200)" % (
-        format(w.Tq, ","), format(w.Tkv, ","), w.B, w.H, w.D)
+    return "quantized attention%s effective TOPS and ms/call at Tq=%s, Tkv=%s, B=%d, H=%d, D=%d (1xB200)" % (
+        " with Q/K RMSNorm + RoPE" if w.norm_rope else "", format(w.Tq, ","), format(w.Tkv, ","), w.B, w.H, w.D)
 UNIT = "TOPS"
 DEFAULT_WORKLOAD = "h3_t37810_h32"
 KERNEL_SOURCES = ["quantized_attention_video_b200/csrc/attention.cu", "quantized_attention_video_b200/csrc/sm100_ptx.cuh"]
@@ -70,7 +70,9 @@ def dist_env():
 def config_of(w: synth.Workload, world: int) -> dict:
     return {"workload": w.name, "B": w.B, "Tq": w.Tq, "Tkv": w.Tkv, "H": w.H, "D": w.D,
             "layout": "packed [B,T,3,H,D] in, [B,T,H*D] out" if w.packed else "separate [B,T,H,D] in and out",
-            "inputs": f"seeded synthetic ({w.recipe}), seed {w.seed}",
+            "inputs": f"seeded synthetic ({w.recipe}), seed {w.seed}" + (
+                "; Q/K RMSNorm + RoPE (gamma ~ N(1, 0.1), eps 1e-6, 3-axis video rotary tables, last 100 tokens "
+                "unrotated) fused into the preparation" if w.norm_rope else ""),
             "l2": "inputs + workspace > 126 MB L2; no flush between steps",
             "parallelism": f"independent replica per GPU x{world}" if world > 1 else "single GPU"}
 
@@ -86,7 +88,10 @@ def cpu_oracle_sample(w: synth.Workload, rows_per_head: int, x=None):
     q, k, v = (x[n][:, :, :1] for n in ("q", "k", "v"))
     threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    z = oracle.quantize(q, k, v)
+    if w.norm_rope:
+        z = oracle.quantize_norm_rope(q, k, v, synth.norm_rope_params(w))
+    else:
+        z = oracle.quantize(q, k, v)
     t_quant = time.perf_counter() - t0
     rng = np.random.default_rng(0)
     if rows_per_head <= 0 or rows_per_head >= w.Tq:
@@ -249,9 +254,20 @@ def run_ours(args, w):
         out = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device=dev)
     ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H, device=dev)
     stream = torch.cuda.current_stream(dev)
+    nr = None
+    if w.norm_rope:
+        nr_host = synth.norm_rope_params(w)
+        nr = {n: torch.from_numpy(np.ascontiguousarray(nr_host[n])).to(dev) for n in h3.NORM_ROPE_FIELDS}
+        nr["eps"] = nr_host["eps"]
+
+    def prep():
+        if nr is None:
+            h3.h3attn_quantize_qkv(q, k, v, ws, stream)
+        else:
+            h3.h3attn_quantize_qkv_norm_rope(q, k, v, nr, ws, stream)
 
     def step():
-        h3.h3attn_quantize_qkv(q, k, v, ws, stream)
+        prep()
         h3.h3attn_attend(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, stream)
 
     for _ in range(max(3, args.warmup)):
@@ -269,7 +285,7 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     for i in range(K):
         ev[i][0].record(stream)
-        h3.h3attn_quantize_qkv(q, k, v, ws, stream)
+        prep()
         ev[i][1].record(stream)
         h3.h3attn_attend(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, stream)
         ev[i][2].record(stream)
@@ -289,9 +305,45 @@ def run_ours(args, w):
     attn_avg = max_over_ranks(dist, statistics.mean(attn_ms), dev)
     quant_avg = max_over_ranks(dist, statistics.mean(quant_ms), dev)
 
+    # ------------------------------------------ fused vs separate norm + RoPE
+    norm_rope = None
+    if nr is not None:
+        # the same preparation as a separate norm + RoPE pass over Q and K (written to
+        # scratch tensors) followed by the plain preparation
+        qn, kn = torch.empty_like(q), torch.empty_like(k)
+        ws2 = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H, device=dev)
+
+        def separate():
+            h3.h3attn_norm_rope(q, nr["gamma_q"], nr["cos_q"], nr["sin_q"], nr["eps"], qn, stream)
+            h3.h3attn_norm_rope(k, nr["gamma_k"], nr["cos_k"], nr["sin_k"], nr["eps"], kn, stream)
+
+        for _ in range(3):
+            separate()
+            h3.h3attn_quantize_qkv(qn, kn, v, ws2, stream)
+        Kn = max(5, K // 2)
+        evn = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kn)]
+        torch.cuda.synchronize(dev)
+        for i in range(Kn):
+            evn[i][0].record(stream)
+            separate()
+            evn[i][1].record(stream)
+            h3.h3attn_quantize_qkv(qn, kn, v, ws2, stream)
+            evn[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        sep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evn)
+        plain_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evn)
+        norm_rope = {"fused_prep_ms": max_over_ranks(dist, statistics.mean(quant_ms), dev),
+                     "separate_pass_ms": max_over_ranks(dist, sep_ms, dev),
+                     "plain_prep_ms": max_over_ranks(dist, plain_ms, dev),
+                     "separate_pass_gbs": 4.0 * (w.Tq + w.Tkv) * w.B * w.H * w.D / (sep_ms * 1e-3) / 1e9,
+                     "note": "fused = h3attn_quantize_qkv_norm_rope; separate = h3attn_norm_rope on Q and K "
+                             "(read + write 2 B each, plus 2 x 256 B of tables per token) then h3attn_quantize_qkv"}
+        if h3.h3attn_check_status(ws2, stream) != h3.OK:
+            raise RuntimeError("device status not OK in the separate-pass timing")
+
     # ------------------------------------------------ end to end (host buffers)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and nr is None:
         # pinned host inputs and output; the library uploads, computes and downloads
         # head groups on overlapping streams (h3attn_forward_host)
         if w.packed:
@@ -365,6 +417,9 @@ def run_ours(args, w):
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic", "config": config_of(w, world),
             "clocks": clk, "gpu_launches": 4 * K, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu}
+    if norm_rope is not None:
+        line["norm_rope"] = norm_rope
+        line["e2e_note"] = "the host-buffer pipeline has no norm + RoPE variant; e2e is measured on the plain workloads"
     print(json.dumps(line), flush=True)
 
 

@@ -241,6 +241,55 @@ h3attn_status h3attn_forward_static(const h3attn_bf16_view* q, const h3attn_bf16
                                     const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
                                     float softmax_scale, const h3attn_bf16_out* out, void* stream);
 
+/* ---- Q/K RMSNorm + RoPE before the attention ("H3 Performance Roadmap", Component 2
+ * execution order, item 1: Q/K normalization and RoPE where the attention consumes Q
+ * and K; "Norm and RoPE" in the representative block table).  The pages give no
+ * formula; the one implemented, per (b, t, h) row of 128 channels x:
+ *   ss  = sum of x_c^2 in FP32 (sixteen 8-channel slice sums, each in channel order,
+ *         then added pairwise: slice s += slice s+8 for s < 8, then s += s+4 for s < 4,
+ *         s += s+2, s += s+1; every product and sum rounded separately);
+ *   r   = 1 / sqrt(ss / 128 + eps)   (FP32; sqrt and division correctly rounded);
+ *   z_c = bf16(bf16(x_c * r) * gamma_c);
+ *   out_2i   = bf16(z_2i * cos_i - z_2i+1 * sin_i),
+ *   out_2i+1 = bf16(z_2i+1 * cos_i + z_2i * sin_i)  (FP32, every product and sum rounded,
+ *                                                     no fused multiply-add).
+ * Positions are the caller's: row t of the cos/sin tables belongs to token t of every
+ * batch item and head (a 3-axis video RoPE, or cos 1 / sin 0 for tokens left
+ * unrotated, is encoded in the tables). */
+typedef struct {
+  const float* gamma_q; /* [128] FP32 RMSNorm weight applied to Q (device, 16-byte aligned) */
+  const float* gamma_k; /* [128] FP32 weight applied to K */
+  const float* cos_q;   /* [Tq, 64] FP32 rotary tables of the query positions (row-major, */
+  const float* sin_q;   /*          device, 16-byte aligned) */
+  const float* cos_k;   /* [Tkv, 64] FP32 rotary tables of the key positions */
+  const float* sin_k;
+  float eps;            /* > 0 and finite */
+} h3attn_qk_norm_rope;
+
+/* h3attn_quantize_qkv on the normalized and rotated Q and K: every Q and K row goes
+ * through the transform above in registers as the preparation kernels load it (V
+ * unchanged), so the words are bit for bit those of h3attn_norm_rope on Q and K
+ * followed by h3attn_quantize_qkv, without the separate pass's HBM round trip.
+ * H3ATTN_ERR_INVALID_ARG for a null nr or table, or eps not > 0 and finite;
+ * H3ATTN_ERR_ALIGNMENT for a table not 16-byte aligned. */
+h3attn_status h3attn_quantize_qkv_norm_rope(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                            const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                            const h3attn_qk_norm_rope* nr, void* ws, size_t ws_bytes,
+                                            void* stream);
+
+/* h3attn_quantize_qkv_norm_rope + h3attn_attend. */
+h3attn_status h3attn_forward_norm_rope(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                       const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                       float softmax_scale, const h3attn_qk_norm_rope* nr,
+                                       const h3attn_bf16_out* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The transform above as a separate pass: x [B, T, H, 128] -> out (same shape, any
+ * strides).  gamma [128], cos/sin [T, 64]: FP32 device arrays, 16-byte aligned.  out
+ * may be x itself (in place); partially overlapping views are undefined. */
+h3attn_status h3attn_norm_rope(const h3attn_bf16_view* x, int B, int T, int H, int D, const float* gamma,
+                               const float* cos_tab, const float* sin_tab, float eps,
+                               const h3attn_bf16_out* out, void* stream);
+
 /* Static description of a status code. */
 const char* h3attn_status_string(h3attn_status s);
 

@@ -36,6 +36,14 @@ class _View(ctypes.Structure):
                 ("stride_h", ctypes.c_int64)]
 
 
+class _NormRope(ctypes.Structure):
+    _fields_ = [("gamma_q", ctypes.c_void_p), ("gamma_k", ctypes.c_void_p), ("cos_q", ctypes.c_void_p),
+                ("sin_q", ctypes.c_void_p), ("cos_k", ctypes.c_void_p), ("sin_k", ctypes.c_void_p),
+                ("eps", ctypes.c_float)]
+
+
+NORM_ROPE_FIELDS = ("gamma_q", "gamma_k", "cos_q", "sin_q", "cos_k", "sin_k")
+
 _lib = None
 
 
@@ -76,6 +84,13 @@ def lib() -> ctypes.CDLL:
         L.h3attn_forward_host.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, I, P, S, P]
         L.h3attn_forward_host_check_status.restype = I
         L.h3attn_forward_host_check_status.argtypes = [P] + [I] * 6 + [P]
+        NP = ctypes.POINTER(_NormRope)
+        L.h3attn_quantize_qkv_norm_rope.restype = I
+        L.h3attn_quantize_qkv_norm_rope.argtypes = [VP, VP, VP] + [I] * 5 + [NP, P, S, P]
+        L.h3attn_forward_norm_rope.restype = I
+        L.h3attn_forward_norm_rope.argtypes = [VP, VP, VP] + [I] * 5 + [F, NP, VP, P, S, P]
+        L.h3attn_norm_rope.restype = I
+        L.h3attn_norm_rope.argtypes = [VP] + [I] * 4 + [P, P, P, F, VP, P]
         L.h3attn_status_string.restype = ctypes.c_char_p
         L.h3attn_status_string.argtypes = [I]
         L.h3attn_version.restype = I
@@ -170,6 +185,54 @@ def h3attn_forward(q, k, v, softmax_scale: float, out, ws, stream=None):
     vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
     _check(lib().h3attn_forward(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, T, H, D, softmax_scale,
                                 ctypes.byref(vo), wp, wb, _stream(stream)), "h3attn_forward")
+
+
+def _table(t, n: int, where: str) -> int:
+    """Device pointer of a contiguous FP32 CUDA tensor with n elements."""
+    import torch
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() != n:
+        raise ValueError(f"{where}: expected a contiguous float32 CUDA tensor of {n} elements")
+    return t.data_ptr()
+
+
+def _norm_rope(nr: dict, Tq: int, Tkv: int, D: int) -> _NormRope:
+    """nr: gamma_q, gamma_k [D]; cos_q, sin_q [Tq, D/2]; cos_k, sin_k [Tkv, D/2] (FP32 CUDA); eps."""
+    sizes = dict(gamma_q=D, gamma_k=D, cos_q=Tq * D // 2, sin_q=Tq * D // 2, cos_k=Tkv * D // 2,
+                 sin_k=Tkv * D // 2)
+    return _NormRope(*(_table(nr[f], sizes[f], f) for f in NORM_ROPE_FIELDS), float(nr["eps"]))
+
+
+def h3attn_quantize_qkv_norm_rope(q, k, v, nr: dict, ws, stream=None):
+    """h3attn_quantize_qkv with the Q/K RMSNorm + RoPE applied as the rows are loaded."""
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(ws)
+    vq, vk, vv = _view(q), _view(k), _view(v)
+    n = _norm_rope(nr, Tq, Tkv, D)
+    _check(lib().h3attn_quantize_qkv_norm_rope(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H,
+                                               D, ctypes.byref(n), wp, wb, _stream(stream)),
+           "h3attn_quantize_qkv_norm_rope")
+
+
+def h3attn_forward_norm_rope(q, k, v, softmax_scale: float, nr: dict, out, ws, stream=None):
+    """Quantize (with the Q/K RMSNorm + RoPE) + attend."""
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(ws)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    n = _norm_rope(nr, Tq, Tkv, D)
+    _check(lib().h3attn_forward_norm_rope(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv, H, D,
+                                          softmax_scale, ctypes.byref(n), ctypes.byref(vo), wp, wb, _stream(stream)),
+           "h3attn_forward_norm_rope")
+
+
+def h3attn_norm_rope(x, gamma, cos_tab, sin_tab, eps: float, out, stream=None):
+    """The separate RMSNorm + RoPE pass: x, out [B, T, H, 128] BF16 views (out may be x)."""
+    B, T, H, D = x.shape
+    vx, vo = _view(x), _view(out)
+    _check(lib().h3attn_norm_rope(ctypes.byref(vx), B, T, H, D, _table(gamma, D, "gamma"),
+                                  _table(cos_tab, T * D // 2, "cos"), _table(sin_tab, T * D // 2, "sin"), eps,
+                                  ctypes.byref(vo), _stream(stream)), "h3attn_norm_rope")
 
 
 def h3attn_forward_host_bytes(B: int, Tq: int, Tkv: int, H: int, heads_per_group: int, D: int = HEAD_DIM) -> int:

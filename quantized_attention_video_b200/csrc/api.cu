@@ -38,6 +38,13 @@ h3attn_status check_out(const h3attn_bf16_out* o) {
   return check_strides(o->data, o->stride_b, o->stride_t, o->stride_h);
 }
 
+// An FP32 parameter table (gamma, cos, sin): non-null, 16-byte aligned (float4 loads).
+h3attn_status check_table(const float* t) {
+  if (t == nullptr) return H3ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(t) % 16 != 0) return H3ATTN_ERR_ALIGNMENT;
+  return H3ATTN_OK;
+}
+
 h3attn_status check_ws(const void* ws, size_t bytes, const Layout& L) {
   if (ws == nullptr) return H3ATTN_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return H3ATTN_ERR_WORKSPACE;
@@ -132,6 +139,54 @@ h3attn_status h3attn_forward(const h3attn_bf16_view* q, const h3attn_bf16_view* 
                              int B, int T, int H, int D, float softmax_scale, const h3attn_bf16_out* out, void* ws,
                              size_t ws_bytes, void* stream) {
   return h3attn_forward_ex(q, k, v, B, T, T, H, D, softmax_scale, out, ws, ws_bytes, stream);
+}
+
+h3attn_status h3attn_quantize_qkv_norm_rope(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                            const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                            const h3attn_qk_norm_rope* nr, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  H3_TRY(check_sizes(B, Tq, Tkv, H, D));
+  H3_TRY(check_view(q));
+  H3_TRY(check_view(k));
+  H3_TRY(check_view(v));
+  if (nr == nullptr) return H3ATTN_ERR_INVALID_ARG;
+  for (const float* t : {nr->gamma_q, nr->gamma_k, nr->cos_q, nr->sin_q, nr->cos_k, nr->sin_k})
+    H3_TRY(check_table(t));
+  if (!(nr->eps > 0.0f) || !std::isfinite(nr->eps)) return H3ATTN_ERR_INVALID_ARG;
+  const Shape s = make_shape(B, Tq, Tkv, H);
+  const Layout L = make_layout(s);
+  H3_TRY(check_ws(ws, ws_bytes, L));
+  H3_TRY(check_device());
+  if (launch_quantize(*q, *k, *v, s, L, static_cast<char*>(ws), static_cast<cudaStream_t>(stream), nr) !=
+      cudaSuccess)
+    return H3ATTN_ERR_CUDA;
+  return H3ATTN_OK;
+}
+
+h3attn_status h3attn_forward_norm_rope(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                       const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                       float softmax_scale, const h3attn_qk_norm_rope* nr,
+                                       const h3attn_bf16_out* out, void* ws, size_t ws_bytes, void* stream) {
+  H3_TRY(check_sizes(B, Tq, Tkv, H, D));
+  H3_TRY(check_out(out));
+  if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return H3ATTN_ERR_INVALID_ARG;
+  H3_TRY(h3attn_quantize_qkv_norm_rope(q, k, v, B, Tq, Tkv, H, D, nr, ws, ws_bytes, stream));
+  return h3attn_attend(ws, ws_bytes, B, Tq, Tkv, H, D, softmax_scale, out, stream);
+}
+
+h3attn_status h3attn_norm_rope(const h3attn_bf16_view* x, int B, int T, int H, int D, const float* gamma,
+                               const float* cos_tab, const float* sin_tab, float eps,
+                               const h3attn_bf16_out* out, void* stream) {
+  H3_TRY(check_sizes(B, T, T, H, D));
+  H3_TRY(check_view(x));
+  H3_TRY(check_out(out));
+  for (const float* t : {gamma, cos_tab, sin_tab}) H3_TRY(check_table(t));
+  if (!(eps > 0.0f) || !std::isfinite(eps)) return H3ATTN_ERR_INVALID_ARG;
+  H3_TRY(check_device());
+  if (launch_norm_rope(*x, B, T, H, gamma, cos_tab, sin_tab, eps, *out, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return H3ATTN_ERR_CUDA;
+  return H3ATTN_OK;
 }
 
 h3attn_status h3attn_check_status(void* ws, void* stream) {

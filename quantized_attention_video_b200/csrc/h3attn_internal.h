@@ -77,8 +77,13 @@ struct DevStatus {
 };
 
 // Kernel launchers (defined in quantize.cu / attention.cu).
+// nr != nullptr: Q and K rows pass through the RMSNorm + RoPE transform as they are loaded.
 cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
-                            const Shape& s, const Layout& L, char* ws, cudaStream_t st);
+                            const Shape& s, const Layout& L, char* ws, cudaStream_t st,
+                            const h3attn_qk_norm_rope* nr = nullptr);
+// The separate RMSNorm + RoPE pass over a [B, T, H, 128] view.
+cudaError_t launch_norm_rope(const h3attn_bf16_view& x, int B, int T, int H, const float* gamma, const float* cosv,
+                             const float* sinv, float eps, const h3attn_bf16_out& out, cudaStream_t st);
 
 // The attention grid: one CTA per pair of 128-row Q tiles of one (b, h).
 inline int64_t attention_ctas(const Shape& s) { return ((s.Tq_pad / kTile + 1) / 2) * (int64_t)s.H * s.B; }

@@ -22,6 +22,16 @@
 //
 // All loads are 16-byte vectors of 8 BF16 channels; 16 threads cover one
 // 128-channel row, so a warp reads two contiguous 256-byte rows per load.
+//
+// With the Q/K RMSNorm + RoPE preparation ("H3 Performance Roadmap", Component 2
+// item 1: Q/K normalization and RoPE where the attention consumes Q and K), each
+// Q and K row passes through norm_rope_row once, in registers, so the
+// quantization sees the same BF16 values a separate norm_rope_kernel pass would
+// have written.  norm_rope_kernel writes the transformed Q straight into the
+// Q-word area of the workspace; the statistics pass transforms K (it needs it for
+// the K means) and leaves it in the K-word area; the quantize pass reads both from
+// there and overwrites them with the words.  Q, K and V are read raw once, and K
+// is never written or re-read outside the workspace.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -48,6 +58,97 @@ __device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
+// ------------------------------------------------------- Q/K norm + RoPE ----
+// Two FP32 values rounded to the nearest BF16 (ties to even) and packed, lo in the low half.
+__device__ __forceinline__ uint32_t bf16_pair(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// a, b replaced by their values rounded to the nearest BF16.
+__device__ __forceinline__ void bf16_round2(float& a, float& b) {
+  const uint32_t u = bf16_pair(a, b);
+  a = __uint_as_float(u << 16);
+  b = __uint_as_float(u & 0xFFFF0000u);
+}
+
+// The half-warp of this thread (the 16 lanes that share one row).
+__device__ __forceinline__ unsigned half_warp_mask() { return 0xFFFFu << (threadIdx.x & 16); }
+
+// Per-head RMSNorm and rotary embedding of 128-channel rows.  The 16 lanes of a
+// half-warp (lane & 15 = c16) hold channels [8 c16, 8 c16 + 8) of a row as one
+// 16-byte word each and get them back transformed:
+//   ss  = sum of x^2 in FP32: each lane adds its 8 squares in channel order, then
+//         the 16 slice sums are added pairwise over lane distances 8, 4, 2, 1
+//         (slice s with s + 8, those pairs with the pairs 4 apart, ...);
+//   r   = 1 / sqrt(ss / 128 + eps), each FP32 step correctly rounded;
+//   z_c = bf16(bf16(x_c r) * gamma_c);
+//   (z_2i, z_2i+1) rotated by (cos_i, sin_i), every product and sum rounded to
+//   FP32 separately (no FMA), then to BF16.
+// Every product that feeds a sum uses the __fmul_rn / __fadd_rn intrinsics, which
+// the compiler never contracts into a fused multiply-add (packed FP32-pair
+// arithmetic gave fused results for the rotation in a measured build).  Each sum
+// of the tree is computed by the lanes of its two operands with the operands
+// swapped; addition commutes, so they get the same bits.
+
+// This lane's 8 squares, in channel order.
+__device__ __forceinline__ float slice_ss(const float (&x)[8]) {
+  float part = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part = __fadd_rn(part, __fmul_rn(x[e], x[e]));
+  return part;
+}
+
+// 1 / sqrt(ss / 128 + eps).
+__device__ __forceinline__ float rms_rcp(float ss, float eps) {
+  const float ms = __fmul_rn(ss, 1.0f / kD);  // exact scaling: the same value as ss / 128
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+}
+
+// n, z and the rotation of this lane's channels given r; g holds gamma of them, c
+// and sn cos/sin of pairs [4 c16, 4 c16 + 4).
+__device__ __forceinline__ uint4 norm_rope_apply(const float (&x)[8], float r, const float (&g)[8], float4 c,
+                                                 float4 sn) {
+  const uint64_t rr = f2_pack(r, r);
+  const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {sn.x, sn.y, sn.z, sn.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a, b;
+    f2_unpack(f2_mul(f2_pack(x[2 * i], x[2 * i + 1]), rr), a, b);
+    bf16_round2(a, b);  // n
+    f2_unpack(f2_mul(f2_pack(a, b), f2_pack(g[2 * i], g[2 * i + 1])), a, b);
+    bf16_round2(a, b);  // z
+    // (a c - b s, b c + a s): products rounded, then one rounded sum each
+    o[i] = bf16_pair(__fsub_rn(__fmul_rn(a, cc[i]), __fmul_rn(b, ss[i])),
+                     __fadd_rn(__fmul_rn(b, cc[i]), __fmul_rn(a, ss[i])));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// One row per half-warp (`mask`): cs, sn point at cos/sin of pairs [4 c16, 4 c16 + 4)
+// of the row's token (16-byte aligned).
+__device__ __forceinline__ uint4 norm_rope_row(uint4 w, const float (&g)[8], const float* cs, const float* sn,
+                                               float eps, unsigned mask) {
+  const float4 c = __ldg(reinterpret_cast<const float4*>(cs));
+  const float4 s = __ldg(reinterpret_cast<const float4*>(sn));
+  float x[8];
+  unpack8(w, x);
+  float part = slice_ss(x);
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(mask, part, o));
+  return norm_rope_apply(x, rms_rcp(part, eps), g, c, s);
+}
+
+// gamma of channels [8 c16, 8 c16 + 8)
+__device__ __forceinline__ void load_gamma8(const float* gamma, int c16, float (&g)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(gamma + 8 * c16));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(gamma + 8 * c16 + 4));
+  g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w;
+  g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
+}
+
+
 // All three kernels take the same arguments.
 struct PrepParams {
   const uint16_t* q;
@@ -68,10 +169,20 @@ struct PrepParams {
   float* sk;
   uint8_t* v8t;
   DevStatus* status;
+  // Q/K RMSNorm + RoPE (kNormRope instantiations only): gamma [128], cos/sin [T, 64]
+  const float* gamma_q;
+  const float* gamma_k;
+  const float* cos_q;
+  const float* sin_q;
+  const float* cos_k;
+  const float* sin_k;
+  float eps;
 };
 
 // ------------------------------------------------------------------ stats ----
-// One (unit, sub) pair: unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice.
+// One (unit, sub) pair: unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice; the 16
+// subs of a unit are the 16 lanes of one half-warp.
+template <bool kNormRope>
 __device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, int sub) {
   const int64_t chunk = unit % p.nchunk, bh = unit / p.nchunk;
   const int64_t h = bh % p.H, b = bh / p.H;
@@ -81,12 +192,20 @@ __device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, in
   const uint16_t* vp = p.v + b * p.vsb + h * p.vsh + sub * 8;
   double acc[8];
   float vm[8];
+  float g[8];
+  if (kNormRope) load_gamma8(p.gamma_k, sub, g);
 #pragma unroll
   for (int e = 0; e < 8; ++e) { acc[e] = 0.0; vm[e] = 0.0f; }
 #pragma unroll 4
   for (int t = t0; t < t1; ++t) {
     float kf[8], vf[8];
-    unpack8(ldg16(kp + (int64_t)t * p.kst), kf);
+    uint4 kw = ldg16(kp + (int64_t)t * p.kst);
+    if (kNormRope) {
+      kw = norm_rope_row(kw, g, p.cos_k + (int64_t)t * (kD / 2) + 4 * sub, p.sin_k + (int64_t)t * (kD / 2) + 4 * sub,
+                         p.eps, half_warp_mask());
+      *reinterpret_cast<uint4*>(p.k8 + (bh * p.Tkv_pad + t) * kD + sub * 8) = kw;
+    }
+    unpack8(kw, kf);
     unpack8(ldg16(vp + (int64_t)t * p.vst), vf);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -108,6 +227,7 @@ __device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, in
 // order).  The same sums and maxima as stats_unit.
 constexpr int kStatsThreads = 256;
 
+template <bool kNormRope>
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p) {
   __shared__ __align__(16) uint16_t ks[kTile * kD];                 // [row][channel] BF16
   __shared__ float vred[kStatsThreads / 32][kTile / kChunk][kD];  // [warp][chunk][channel]
@@ -124,6 +244,20 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p
     const bool in = t < p.Tkv;
     kr[i] = in ? ldg16(kp + t * p.kst) : make_uint4(0u, 0u, 0u, 0u);
     vr[i] = in ? ldg16(vp + t * p.vst) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (kNormRope) {
+    // the slab's K rows, transformed; also left in the K-word area for the quantize pass
+    float g[8];
+    load_gamma8(p.gamma_k, c16, g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t t = t0 + r0 + 16 * i;
+      if (t < p.Tkv) {  // the same for the 16 lanes of the row
+        kr[i] = norm_rope_row(kr[i], g, p.cos_k + t * (kD / 2) + 4 * c16, p.sin_k + t * (kD / 2) + 4 * c16, p.eps,
+                              half_warp_mask());
+        *reinterpret_cast<uint4*>(p.k8 + (bh * p.Tkv_pad + t) * kD + c16 * 8) = kr[i];
+      }
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(ks + (r0 + 16 * i) * kD + c16 * 8) = kr[i];
@@ -298,7 +432,19 @@ __device__ __forceinline__ void load_rows(uint4 (&raw)[8], const uint16_t* p, in
   }
 }
 
+// load_rows from a dense [T_pad, 128] row block written earlier (by another kernel,
+// or by this block before a barrier): loads cached in L2 only, never the
+// non-coherent read-only path.
+__device__ __forceinline__ void load_rows_cg(uint4 (&raw)[8], const uint16_t* p, int64_t t0, int rq, int T) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int64_t t = t0 + 8 * rq + r;
+    raw[r] = t < T ? __ldcg(reinterpret_cast<const uint4*>(p + t * kD)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 // Slab `slab` (128 tokens) of (b, h).  red, gmax and vt are the block's shared scratch.
+template <bool kNormRope>
 __device__ __forceinline__ void quantize_slab(const PrepParams& p, int64_t slab, int64_t h, int64_t b, float* red,
                                               float* gmax, uint8_t* vt) {
   const uint16_t* __restrict__ q = p.q;
@@ -324,8 +470,14 @@ __device__ __forceinline__ void quantize_slab(const PrepParams& p, int64_t slab,
 
   // padding rows (t >= T) load as zero words (BF16 +0)
   uint4 rq8[8], rk8[8], rv8[8];
-  load_rows(rq8, q + b * qsb + h * qsh + c16 * 8, qst, t0, rq, has_q ? Tq : 0);
-  load_rows(rk8, k + b * ksb + h * ksh + c16 * 8, kst, t0, rq, has_kv ? Tkv : 0);
+  if (kNormRope) {
+    // Q and K rows already transformed by the statistics pass, in this slab's word areas
+    load_rows_cg(rq8, p.q8 + bh * Tq_pad * kD + c16 * 8, t0, rq, has_q ? Tq : 0);
+    load_rows_cg(rk8, p.k8 + bh * Tkv_pad * kD + c16 * 8, t0, rq, has_kv ? Tkv : 0);
+  } else {
+    load_rows(rq8, q + b * qsb + h * qsh + c16 * 8, qst, t0, rq, has_q ? Tq : 0);
+    load_rows(rk8, k + b * ksb + h * ksh + c16 * 8, kst, t0, rq, has_kv ? Tkv : 0);
+  }
 
   // ---------------------------------------------------------------- Q ----
   if (has_q) {
@@ -449,30 +601,83 @@ __device__ __forceinline__ void quantize_slab(const PrepParams& p, int64_t slab,
 
 
 // Slab blockIdx.x of (b = blockIdx.z, h = blockIdx.y).
+template <bool kNormRope>
 __global__ void __launch_bounds__(256, 2) quantize_kernel(const PrepParams p) {
   __shared__ float red[8];
   __shared__ float gmax[4];
   __shared__ __align__(16) uint8_t vt[kD * kTile];  // [channel][token], 16-byte chunks XOR-swizzled
-  quantize_slab(p, blockIdx.x, blockIdx.y, blockIdx.z, red, gmax, vt);
+  quantize_slab<kNormRope>(p, blockIdx.x, blockIdx.y, blockIdx.z, red, gmax, vt);
 }
 
 // Short sequences: the whole preparation of (b, h) = blockIdx.x in one block and one
 // launch (statistics, their ordered reduction, then every slab), the same arithmetic
 // as the three-kernel path.  Every stage's global writes are read by other threads of
 // the block only after a block barrier.
+template <bool kNormRope>
 __global__ void __launch_bounds__(256, 1) prep_small_kernel(const PrepParams p) {
   __shared__ float red[8];
   __shared__ float gmax[4];
   __shared__ __align__(16) uint8_t vt[kD * kTile];
   const int64_t bh = blockIdx.x;
   if (bh == 0 && threadIdx.x == 0) clear_status(p);
+  if (kNormRope) {
+    // Q rows transformed into the Q-word area (half-warp = one row), K rows by stats_unit
+    const int c16 = threadIdx.x & 15;
+    float g[8];
+    load_gamma8(p.gamma_q, c16, g);
+    const uint16_t* qp = p.q + (bh / p.H) * p.qsb + (bh % p.H) * p.qsh + c16 * 8;
+    for (int64_t t = threadIdx.x >> 4; t < p.Tq; t += blockDim.x >> 4)
+      *reinterpret_cast<uint4*>(p.q8 + (bh * p.Tq_pad + t) * kD + c16 * 8) =
+          norm_rope_row(ldg16(qp + t * p.qst), g, p.cos_q + t * (kD / 2) + 4 * c16, p.sin_q + t * (kD / 2) + 4 * c16,
+                        p.eps, half_warp_mask());
+  }
   for (int64_t c = threadIdx.x >> 4; c < p.nchunk; c += blockDim.x >> 4)
-    stats_unit(p, bh * p.nchunk + c, (int)(threadIdx.x & 15));
+    stats_unit<kNormRope>(p, bh * p.nchunk + c, (int)(threadIdx.x & 15));
   __syncthreads();
   if (threadIdx.x < kD) finalize_channel(p, bh, threadIdx.x);
   __syncthreads();
   const int64_t slabs = (p.Tq_pad > p.Tkv_pad ? p.Tq_pad : p.Tkv_pad) / kTile;
-  for (int64_t slab = 0; slab < slabs; ++slab) quantize_slab(p, slab, bh % p.H, bh / p.H, red, gmax, vt);
+  for (int64_t slab = 0; slab < slabs; ++slab) quantize_slab<kNormRope>(p, slab, bh % p.H, bh / p.H, red, gmax, vt);
+}
+
+// Separate Q/K RMSNorm + RoPE pass (BF16 in, BF16 out) over the (b, t, h) rows of the
+// [B, T, H, 128] view x: each half-warp takes kNormRopeRows consecutive rows, loads
+// them all before transforming any, and writes them to the same rows of out.  out
+// may be x itself (each lane reads its 16 bytes of a row before writing them).  The
+// fused preparation also runs it on Q with out = the Q-word area of the workspace.
+constexpr int kNormRopeRows = 4;
+
+__global__ void __launch_bounds__(256) norm_rope_kernel(const uint16_t* x, int64_t xsb, int64_t xst, int64_t xsh,
+                                                        uint16_t* out, int64_t osb, int64_t ost, int64_t osh, int T,
+                                                        int H, int64_t nrows, const float* gamma, const float* cosv,
+                                                        const float* sinv, float eps) {
+  const int64_t row0 = ((int64_t)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4)) * kNormRopeRows;
+  const int c16 = threadIdx.x & 15;
+  float g[8];
+  load_gamma8(gamma, c16, g);
+  // (b, t, h) of the first row, then stepped row by row (h fastest)
+  int64_t h = row0 % H, t = (row0 / H) % T, b = row0 / H / T;
+  uint4 w[kNormRopeRows];
+  int64_t oo[kNormRopeRows], tt[kNormRopeRows];
+#pragma unroll
+  for (int j = 0; j < kNormRopeRows; ++j) {
+    oo[j] = b * osb + t * ost + h * osh + c16 * 8;
+    tt[j] = t;
+    w[j] = row0 + j < nrows ? ldg16(x + b * xsb + t * xst + h * xsh + c16 * 8) : make_uint4(0u, 0u, 0u, 0u);
+    if (++h == H) {
+      h = 0;
+      if (++t == T) {
+        t = 0;
+        ++b;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kNormRopeRows; ++j) {
+    if (row0 + j >= nrows) break;  // uniform over the half-warp
+    *reinterpret_cast<uint4*>(out + oo[j]) = norm_rope_row(w[j], g, cosv + tt[j] * (kD / 2) + 4 * c16,
+                                                           sinv + tt[j] * (kD / 2) + 4 * c16, eps, half_warp_mask());
+  }
 }
 
 // The finalize kernel's shared memory is above the default 48 KB limit (set once per device).
@@ -493,7 +698,8 @@ cudaError_t ensure_prep_attrs() {
 }  // namespace
 
 cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k, const h3attn_bf16_view& v,
-                            const Shape& s, const Layout& L, char* ws, cudaStream_t st) {
+                            const Shape& s, const Layout& L, char* ws, cudaStream_t st,
+                            const h3attn_qk_norm_rope* nr) {
   PrepParams p;
   p.q = static_cast<const uint16_t*>(q.data);
   p.qsb = q.stride_b; p.qst = q.stride_t; p.qsh = q.stride_h;
@@ -513,18 +719,53 @@ cudaError_t launch_quantize(const h3attn_bf16_view& q, const h3attn_bf16_view& k
   p.sk = reinterpret_cast<float*>(ws + L.off[H3ATTN_WS_SK]);
   p.v8t = reinterpret_cast<uint8_t*>(ws + L.off[H3ATTN_WS_V8T]);
   p.status = reinterpret_cast<DevStatus*>(ws + L.off[H3ATTN_WS_STATUS]);
+  p.gamma_q = nr ? nr->gamma_q : nullptr;
+  p.gamma_k = nr ? nr->gamma_k : nullptr;
+  p.cos_q = nr ? nr->cos_q : nullptr;
+  p.sin_q = nr ? nr->sin_q : nullptr;
+  p.cos_k = nr ? nr->cos_k : nullptr;
+  p.sin_k = nr ? nr->sin_k : nullptr;
+  p.eps = nr ? nr->eps : 0.0f;
   const int64_t slabs = (s.Tq_pad > s.Tkv_pad ? s.Tq_pad : s.Tkv_pad) / kTile;
   if (slabs <= kSmallSlabs) {
     // few tokens per head: one launch, one block per (b, h)
-    prep_small_kernel<<<(unsigned)((int64_t)s.B * s.H), 256, 0, st>>>(p);
+    if (nr)
+      prep_small_kernel<true><<<(unsigned)((int64_t)s.B * s.H), 256, 0, st>>>(p);
+    else
+      prep_small_kernel<false><<<(unsigned)((int64_t)s.B * s.H), 256, 0, st>>>(p);
     return cudaGetLastError();
   }
   const cudaError_t e = ensure_prep_attrs();
   if (e != cudaSuccess) return e;
-  stats_kernel<<<dim3((unsigned)(s.Tkv_pad / kTile), (unsigned)s.H, (unsigned)s.B), kStatsThreads, 0, st>>>(p);
+  if (nr) {
+    // Q rows transformed by the separate-pass kernel straight into the Q-word area
+    // ([B, H, Tq_pad, 128]), where the quantize pass reads them
+    const h3attn_bf16_out qa = {p.q8, (int64_t)s.H * s.Tq_pad * kD, kD, s.Tq_pad * kD};
+    const cudaError_t e2 = launch_norm_rope(q, s.B, s.Tq, s.H, nr->gamma_q, nr->cos_q, nr->sin_q, nr->eps, qa, st);
+    if (e2 != cudaSuccess) return e2;
+  }
+  const dim3 sgrid((unsigned)(s.Tkv_pad / kTile), (unsigned)s.H, (unsigned)s.B);
+  if (nr)
+    stats_kernel<true><<<sgrid, kStatsThreads, 0, st>>>(p);
+  else
+    stats_kernel<false><<<sgrid, kStatsThreads, 0, st>>>(p);
   finalize_kernel<<<dim3((unsigned)(s.B * s.H), kD / 32), kFinThreads, kFinSmemBytes, st>>>(p);
   dim3 grid((unsigned)slabs, (unsigned)s.H, (unsigned)s.B);
-  quantize_kernel<<<grid, 256, 0, st>>>(p);
+  if (nr)
+    quantize_kernel<true><<<grid, 256, 0, st>>>(p);
+  else
+    quantize_kernel<false><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_rope(const h3attn_bf16_view& x, int B, int T, int H, const float* gamma, const float* cosv,
+                             const float* sinv, float eps, const h3attn_bf16_out& out, cudaStream_t st) {
+  const int64_t nrows = (int64_t)B * T * H;
+  const int64_t per_block = 16 * kNormRopeRows;
+  const int64_t blocks = (nrows + per_block - 1) / per_block;
+  norm_rope_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const uint16_t*>(x.data), x.stride_b, x.stride_t, x.stride_h, static_cast<uint16_t*>(out.data),
+      out.stride_b, out.stride_t, out.stride_h, T, H, nrows, gamma, cosv, sinv, eps);
   return cudaGetLastError();
 }
 

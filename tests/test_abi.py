@@ -118,6 +118,41 @@ def test_host_pipeline_sizes_and_argument_errors(L):
     assert args(nbytes=1000) == h3.ERR_WORKSPACE
 
 
+def test_norm_rope_argument_errors(L):
+    good = _view(0x100000)
+    tab = 0x5000000
+
+    def nr(**kw):
+        f = dict(gamma_q=tab, gamma_k=tab, cos_q=tab, sin_q=tab, cos_k=tab, sin_k=tab, eps=1e-6)
+        f.update(kw)
+        return h3._NormRope(*(f[n] for n in h3.NORM_ROPE_FIELDS), f["eps"])
+
+    def fwd(n, D=128):
+        return L.h3attn_forward_norm_rope(ctypes.byref(good), ctypes.byref(good), ctypes.byref(good), 1, 256, 256, 4,
+                                          D, 0.088, ctypes.byref(n) if n is not None else None,
+                                          ctypes.byref(_view(0x2000000)), 0x1000000, 1 << 40, None)
+
+    assert fwd(None) == h3.ERR_INVALID_ARG
+    assert fwd(nr(), D=64) == h3.ERR_UNSUPPORTED
+    assert fwd(nr(cos_k=0)) == h3.ERR_INVALID_ARG
+    assert fwd(nr(gamma_q=tab + 4)) == h3.ERR_ALIGNMENT
+    assert fwd(nr(eps=0.0)) == h3.ERR_INVALID_ARG
+    assert fwd(nr(eps=float("inf"))) == h3.ERR_INVALID_ARG
+    q = L.h3attn_quantize_qkv_norm_rope
+    assert q(ctypes.byref(good), ctypes.byref(good), ctypes.byref(good), 1, 256, 256, 4, 128, None, 0x1000000,
+             1 << 40, None) == h3.ERR_INVALID_ARG
+    assert q(ctypes.byref(good), ctypes.byref(good), ctypes.byref(good), 1, 256, 256, 4, 128, ctypes.byref(nr()), 0,
+             1 << 40, None) == h3.ERR_WORKSPACE
+    f = L.h3attn_norm_rope
+    out = _view(0x2000000)
+    assert f(ctypes.byref(good), 1, 256, 4, 128, tab, tab, 0, 1e-6, ctypes.byref(out), None) == h3.ERR_INVALID_ARG
+    assert f(ctypes.byref(good), 1, 256, 4, 128, tab, tab + 8, tab, 1e-6, ctypes.byref(out), None) == h3.ERR_ALIGNMENT
+    assert f(ctypes.byref(good), 1, 256, 4, 128, tab, tab, tab, -1.0, ctypes.byref(out), None) == h3.ERR_INVALID_ARG
+    assert f(ctypes.byref(_view(0x100004)), 1, 256, 4, 128, tab, tab, tab, 1e-6, ctypes.byref(out),
+             None) == h3.ERR_ALIGNMENT
+    assert f(ctypes.byref(good), 1, 0, 4, 128, tab, tab, tab, 1e-6, ctypes.byref(out), None) == h3.ERR_INVALID_ARG
+
+
 def test_product_path_has_no_oracle_or_cpu_fallback():
     pkg = os.path.join(ROOT, "quantized_attention_video_b200")
     for dirpath, _, files in os.walk(pkg):
