@@ -82,6 +82,23 @@ def test_fused_preparation_and_forward(B, Tq, Tkv, H):
     compare_out(bits(out4), oracle.attend_all(z, w.scale, EPOCH), w.name)
 
 
+def test_fused_reads_packed_strided_views():
+    # raw Q/K/V read in place from one packed [B, T, 3, H, D] buffer, output into [B, T, H*D]
+    w = synth.Workload("nr_packed_b2", 2, 300, 300, 3, 128, "normal", 4301, packed=True, norm_rope=True)
+    x = synth.make_inputs(w)
+    nr = synth.norm_rope_params(w)
+    z = oracle.quantize_norm_rope(x["q"], x["k"], x["v"], nr)
+    d = upload(x, w)
+    dn = dev_params(nr)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    out, out4 = new_out(w)
+    h3.h3attn_forward_norm_rope(d["q"], d["k"], d["v"], w.scale, dn, out4, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    check_quantized(ws, z, w)
+    compare_out(bits(out4), oracle.attend_all(z, w.scale, EPOCH), w.name)
+    assert out.shape == (w.B, w.Tq, w.H * w.D) and out.is_contiguous()
+
+
 def test_bench_shape_fused_equals_oracle_and_separate_pass():
     w = synth.WORKLOADS["h3_t37810_h32_nr"]
     x = synth.make_inputs(w)
