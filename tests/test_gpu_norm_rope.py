@@ -126,3 +126,32 @@ def test_bench_shape_fused_equals_oracle_and_separate_pass():
     vb = h3.workspace_views(ws2, w.B, w.Tq, w.Tkv, w.H)
     for f in ("q8", "k8", "v8t", "sq", "sk", "km", "sv"):
         assert np.array_equal(bits(va[f]), bits(vb[f])), f
+
+
+def test_fused_forward_replays_from_a_cuda_graph():
+    """The norm + RoPE forward (five launches, no host synchronisation) captured once into a
+    CUDA graph replays the bytes of a direct call."""
+    w = synth.WORKLOADS["nr_h4_t1100"]
+    x = synth.make_inputs(w)
+    nr = synth.norm_rope_params(w)
+    d = upload(x, w)
+    dn = dev_params(nr)
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    direct = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    h3.h3attn_forward_norm_rope(d["q"], d["k"], d["v"], w.scale, dn, direct, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    out = torch.zeros_like(direct)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up on the capture stream
+        h3.h3attn_forward_norm_rope(d["q"], d["k"], d["v"], w.scale, dn, out, ws)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        h3.h3attn_forward_norm_rope(d["q"], d["k"], d["v"], w.scale, dn, out, ws)
+    for _ in range(20):
+        out.zero_()
+        g.replay()
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(out.view(torch.int16), direct.view(torch.int16))
+    assert h3.h3attn_check_status(ws) == h3.OK
