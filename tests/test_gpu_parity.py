@@ -354,3 +354,50 @@ def test_forward_replays_from_a_cuda_graph():
         torch.cuda.current_stream().synchronize()
         assert torch.equal(out.view(torch.int16), direct.view(torch.int16))
     assert h3.h3attn_check_status(ws) == h3.OK
+
+
+def test_concurrent_streams_with_separate_workspaces():
+    """Two forward calls in flight at once on two streams, each with its own workspace,
+    give the bytes of the same calls made one after the other (the library keeps no
+    per-call global state)."""
+    wa = synth.Workload("conc_a", 1, 700, 700, 4, 128, "normal", 8101)
+    wb = synth.Workload("conc_b", 2, 333, 900, 3, 128, "k_offset", 8102)
+    runs = []
+    for w in (wa, wb):
+        x = synth.make_inputs(w)
+        d = upload(x, w)
+        ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+        ref = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+        h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, ref, ws)
+        assert h3.h3attn_check_status(ws) == h3.OK
+        runs.append((w, d, h3.new_workspace(w.B, w.Tq, w.Tkv, w.H), ref))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.zeros_like(r[3]) for r in runs]
+    torch.cuda.synchronize()
+    for _ in range(5):
+        for (w, d, ws, _), s, o in zip(runs, streams, outs):
+            h3.h3attn_forward_ex(d["q"], d["k"], d["v"], w.scale, o, ws, stream=s)
+    torch.cuda.synchronize()
+    for (w, d, ws, ref), s, o in zip(runs, streams, outs):
+        assert h3.h3attn_check_status(ws, s) == h3.OK
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16)), w.name
+
+
+def test_random_shapes_against_the_oracle():
+    """A seeded sweep of shapes (batch, ragged lengths, Tq != Tkv, heads, packed or
+    separate layouts): integer stages bit-exact, outputs within tolerance."""
+    rng = np.random.default_rng(20261202)
+    for case in range(8):
+        B = int(rng.integers(1, 3))
+        Tq = int(rng.integers(1, 700))
+        Tkv = Tq if case % 2 == 0 else int(rng.integers(1, 900))
+        H = int(rng.integers(1, 5))
+        packed = case % 2 == 0
+        recipe = ("normal", "k_offset", "rmsnorm")[case % 3]
+        w = synth.Workload(f"rand_{case}", B, Tq, Tkv, H, 128, recipe, 9000 + case, packed=packed)
+        x = synth.make_inputs(w)
+        z = oracle.quantize(x["q"], x["k"], x["v"])
+        d = upload(x, w)
+        ws, out, out4 = run_forward(w, d)
+        check_quantized(ws, z, w)
+        compare_out(bits(out4), oracle.attend_all(z, w.scale, EPOCH), w.name)
