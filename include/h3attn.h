@@ -266,10 +266,13 @@ typedef struct {
   float eps;            /* > 0 and finite */
 } h3attn_qk_norm_rope;
 
-/* h3attn_quantize_qkv on the normalized and rotated Q and K: every Q and K row goes
- * through the transform above in registers as the preparation kernels load it (V
- * unchanged), so the words are bit for bit those of h3attn_norm_rope on Q and K
- * followed by h3attn_quantize_qkv, without the separate pass's HBM round trip.
+/* h3attn_quantize_qkv on the normalized and rotated Q and K (V unchanged).  Four
+ * launches: the transform of Q written straight into the workspace's Q-word area; the
+ * statistics pass, which transforms K in registers (it needs it for the K means) and
+ * leaves it in the K-word area; the ordered reduction; the quantize pass, which reads
+ * Q and K from the workspace and overwrites them with the words.  The words are bit for
+ * bit those of h3attn_norm_rope on Q and K followed by h3attn_quantize_qkv; the raw Q,
+ * K and V are read once and no tensor outside the workspace is written.
  * H3ATTN_ERR_INVALID_ARG for a null nr or table, or eps not > 0 and finite;
  * H3ATTN_ERR_ALIGNMENT for a table not 16-byte aligned. */
 h3attn_status h3attn_quantize_qkv_norm_rope(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
