@@ -169,3 +169,25 @@ def test_rejects_bad_arguments():
     s = np.zeros((2, 64), np.float32)
     with pytest.raises(ValueError):
         oracle.qk_norm_rope(xb, np.ones(D, np.float32), 0.0, c, s)
+
+
+def test_intermediate_roundings_golden():
+    # Hand-derived values that fix the order of the roundings.  Every channel pair of the
+    # row is (+1, -1): mean x^2 = 1; eps = 1.25 gives sqrt(2.25) = 1.5 exactly and
+    # r = RN(1/1.5) = 0.666666686...; n = bf16(r) = 171/256 (the BF16 neighbours are 170/256
+    # and 171/256; r lies above 170.67/256); gamma = 1.25: n*gamma = 855/1024 exactly, which
+    # rounds to z = 214/256 = 0.8359375 (213.75/256).  Without rounding n first, r*1.25 =
+    # 0.83333 rounds to 213/256 instead.
+    #   token 0, cos 1, sin 0: out = (z, -z) = (0.8359375, -0.8359375).
+    #   token 1, cos 0.625, sin 0.5: a*c - b*s = 214/256*5/8 + 214/256/2 = 1926/2048, which
+    #   rounds to 241/256 = 0.94140625 (1926/8 = 240.75); b*c + a*s = -1070/2048 + 856/2048
+    #   = -214/2048 = -0.1044921875 (exact in BF16).  Without rounding z first the first
+    #   value is 7695/8192, which rounds to 240/256 = 0.9375.
+    x = np.tile(np.array([1.0, -1.0], np.float32), 64).reshape(1, 1, 1, D)
+    xb = _bf16(np.concatenate([x, x], axis=1))  # tokens 0 and 1
+    gamma = np.full(D, 1.25, np.float32)
+    cos = np.array([[1.0] * 64, [0.625] * 64], np.float32)
+    sin = np.array([[0.0] * 64, [0.5] * 64], np.float32)
+    got = oracle.bf16_decode(oracle.qk_norm_rope(xb, gamma, 1.25, cos, sin))
+    np.testing.assert_array_equal(got[0, 0, 0], np.tile(np.array([0.8359375, -0.8359375], np.float32), 64))
+    np.testing.assert_array_equal(got[0, 1, 0], np.tile(np.array([0.94140625, -0.1044921875], np.float32), 64))
