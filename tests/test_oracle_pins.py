@@ -214,6 +214,32 @@ def test_scores_equal_integer_matmul():
 
 
 # --------------------------------------------------------------- softmax ----
+def test_dequantized_scores_with_unit_scales():
+    # A closed form of the score path: Q rows hold one channel of value 127 each, K keys
+    # come in +127/-127 pairs per channel, so every K channel mean is exactly 0, every
+    # scale is amax/127 = 1 and the words are the values themselves.  Then acc is in
+    # {16129, -16129, 0} and t = float(acc) * ((sq*sk)*c) reduces to one rounding of
+    # acc * c, with c = float(scale * log2(e)) taken in FP64 and rounded once.
+    D, Tq, Tkv = 128, 5, 10
+    qv = np.zeros((1, Tq, 1, D), np.float32)
+    kv = np.zeros((1, Tkv, 1, D), np.float32)
+    for i in range(Tq):
+        qv[0, i, 0, (3 * i) % 5] = 127.0
+    for j in range(Tkv):
+        kv[0, j, 0, j // 2] = 127.0 if j % 2 == 0 else -127.0
+    vv = np.ones((1, Tkv, 1, D), np.float32)
+    z = oracle.quantize(bf16_bits(qv), bf16_bits(kv), bf16_bits(vv))
+    assert np.all(z["km"] == 0) and np.all(z["sq"] == 1) and np.all(z["sk"] == 1)
+    scale = 0.088388
+    c = np.float32(np.float64(np.float32(scale)) * math.log2(math.e))
+    assert oracle.log2_scale(scale) == c
+    for i in range(Tq):
+        tr = oracle.row_trace(z, scale, 64, 0, 0, i)
+        acc = np.array([16129 * (1 if j % 2 == 0 else -1) if j // 2 == (3 * i) % 5 else 0 for j in range(Tkv)])
+        assert np.array_equal(tr["acc"], acc)
+        assert np.array_equal(tr["t"], (acc.astype(np.float32) * c).astype(np.float32))
+
+
 @pytest.mark.parametrize("epoch", [64, 128])
 def test_softmax_trace_invariants(epoch):
     q, k, v = _qkv(1, 40, 333, 1, 128, seed=17)
