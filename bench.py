@@ -60,6 +60,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same kernel for profiler captures)")
+    ap.add_argument("--latency", action="store_true",
+                    help="per-call latency of the fixed 128 x 192 shape by the pages' method (samples of 20 "
+                         "back-to-back calls, p50 and CV), forward and attend-only samples alternated")
+    ap.add_argument("--samples", type=int, default=500)
     return ap.parse_args()
 
 
@@ -423,8 +427,91 @@ def run_ours(args, w):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------- latency mode ----
+def run_latency(args):
+    """Per-call latency at the fixed shape (B1 H1 Tq128 Tkv192 D128), measured the way the
+    pages measure it ("Phase 2B Aligned Numerical Prototype", the batched p50 over samples
+    of 20 back-to-back launches, with CV): each sample times 20 calls with CUDA events.
+    Forward and attend-only samples alternate in the same process so that clock changes
+    fall on both; a third series replays one CUDA graph of 20 forward calls."""
+    import torch
+    import quantized_attention_video_b200 as h3
+    from quantized_attention_video_b200 import build as h3build
+
+    h3build.build()
+    h3.lib()
+    w = synth.WORKLOADS["fixed_q128_kv192"]
+    x = synth.make_inputs(w)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    q, k, v = dev(x["q"]), dev(x["k"]), dev(x["v"])
+    out = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    per = 20
+
+    def forward():
+        h3.h3attn_forward_ex(q, k, v, w.scale, out, ws)
+
+    def attend():
+        h3.h3attn_attend(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out)
+
+    for _ in range(max(50, args.warmup)):
+        forward()
+    if h3.h3attn_check_status(ws) != h3.OK:
+        raise RuntimeError("device status not OK after warm-up")
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        forward()
+    cur.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(per):
+            forward()
+
+    def sample(run) -> float:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / per
+
+    series = {"forward": [], "attend": [], "graph": []}
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for _ in range(args.samples):
+        series["forward"].append(sample(lambda: [forward() for _ in range(per)]))
+        series["attend"].append(sample(lambda: [attend() for _ in range(per)]))
+        series["graph"].append(sample(graph.replay))
+    clk = clocks.stop()
+    if h3.h3attn_check_status(ws) != h3.OK:
+        raise RuntimeError("device status not OK after the samples")
+
+    def summary(vals):
+        return {"p50_ms": statistics.median(vals), "cv": statistics.pstdev(vals) / statistics.mean(vals)}
+
+    fwd = summary(series["forward"])
+    line = {"metric": "per-call latency, p50 of samples of 20 back-to-back calls, at Tq=128, Tkv=192, B=1, H=1, "
+                      "D=128 (1xB200)",
+            "value": fwd["p50_ms"], "unit": "ms", "higher_is_better": False, "cv": fwd["cv"],
+            "samples": args.samples, "calls_per_sample": per,
+            "attend_only": summary(series["attend"]), "forward_graph_of_20": summary(series["graph"]),
+            "data": "synthetic", "config": dict(config_of(w, 1), l2="the shape's 0.2 MB stays in L2; no flush, as "
+                                                                   "in the pages' method"), "clocks": clk,
+            "note": "forward = h3attn_forward_ex (one preparation launch + the attention launch); samples of "
+                    "the three series interleaved"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.latency:
+        run_latency(args)
+        return
     w = synth.WORKLOADS[args.workload]
     if args.heads:
         import dataclasses
