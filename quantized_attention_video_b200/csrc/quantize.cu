@@ -180,60 +180,21 @@ struct PrepParams {
 };
 
 // ------------------------------------------------------------------ stats ----
-// One (unit, sub) pair: unit = (b*H + h)*nchunk + chunk, sub = 8-channel slice; the 16
-// subs of a unit are the 16 lanes of one half-warp.
-template <bool kNormRope>
-__device__ __forceinline__ void stats_unit(const PrepParams& p, int64_t unit, int sub) {
-  const int64_t chunk = unit % p.nchunk, bh = unit / p.nchunk;
-  const int64_t h = bh % p.H, b = bh / p.H;
-  const int t0 = (int)(chunk * kChunk);
-  const int t1 = min(p.Tkv, t0 + kChunk);
-  const uint16_t* kp = p.k + b * p.ksb + h * p.ksh + sub * 8;
-  const uint16_t* vp = p.v + b * p.vsb + h * p.vsh + sub * 8;
-  double acc[8];
-  float vm[8];
-  float g[8];
-  if (kNormRope) load_gamma8(p.gamma_k, sub, g);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) { acc[e] = 0.0; vm[e] = 0.0f; }
-#pragma unroll 4
-  for (int t = t0; t < t1; ++t) {
-    float kf[8], vf[8];
-    uint4 kw = ldg16(kp + (int64_t)t * p.kst);
-    if (kNormRope) {
-      kw = norm_rope_row(kw, g, p.cos_k + (int64_t)t * (kD / 2) + 4 * sub, p.sin_k + (int64_t)t * (kD / 2) + 4 * sub,
-                         p.eps, half_warp_mask());
-      *reinterpret_cast<uint4*>(p.k8 + (bh * p.Tkv_pad + t) * kD + sub * 8) = kw;
-    }
-    unpack8(kw, kf);
-    unpack8(ldg16(vp + (int64_t)t * p.vst), vf);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc[e] = __dadd_rn(acc[e], (double)kf[e]);
-      vm[e] = fmaxf(vm[e], fabsf(vf[e]));
-    }
-  }
-  double* ko = p.ksum + unit * kD + sub * 8;
-  float* vo = p.vmax + unit * kD + sub * 8;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) { ko[e] = acc[e]; vo[e] = vm[e]; }
-}
-
-// Slab blockIdx.x (128 tokens = chunks 2x, 2x + 1) of (b = blockIdx.z, h = blockIdx.y).
-// Thread (c16 = tid & 15, r0 = tid >> 4) loads channels [8*c16, 8*c16+8) of slab rows
-// r0 + 16 i (i < 8; rows of chunk i / 4): sixteen 16-byte loads in flight per thread.
-// K goes to shared memory, where thread (chunk, channel) then adds its chunk's tokens
-// in token order; the V absmax is reduced from the registers (a max is exact in any
-// order).  The same sums and maxima as stats_unit.
+// Statistics of slab `slab` (128 tokens = chunks 2 slab, 2 slab + 1) of (b, h), by a
+// block of kStatsThreads threads.  Thread (c16 = tid & 15, r0 = tid >> 4) loads channels
+// [8*c16, 8*c16+8) of slab rows r0 + 16 i (i < 8; rows of chunk i / 4): sixteen 16-byte
+// loads in flight per thread.  K goes to shared memory (ks), where thread (chunk,
+// channel) then adds its chunk's tokens in token order in FP64; the V absmax is reduced
+// from the registers (a max is exact in any order) through vred.  Writes the chunk sums
+// and maxima to the ksum / vmax scratch.  Contains one block barrier.
 constexpr int kStatsThreads = 256;
+typedef float VRed[kTile / kChunk][kD];  // [chunk][channel], one per warp
 
 template <bool kNormRope>
-__global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p) {
-  __shared__ __align__(16) uint16_t ks[kTile * kD];                 // [row][channel] BF16
-  __shared__ float vred[kStatsThreads / 32][kTile / kChunk][kD];  // [warp][chunk][channel]
+__device__ __forceinline__ void stats_slab(const PrepParams& p, int64_t slab, int64_t h, int64_t b, uint16_t* ks,
+                                           VRed* vred) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c16 = tid & 15, r0 = tid >> 4;
-  const int64_t slab = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = b * p.H + h, t0 = slab * kTile;
   const uint16_t* kp = p.k + b * p.ksb + h * p.ksh + c16 * 8;
   const uint16_t* vp = p.v + b * p.vsb + h * p.vsh + c16 * 8;
@@ -299,6 +260,14 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p
   const int64_t unit = bh * p.nchunk + chunk;
   p.ksum[unit * kD + ch] = acc;
   p.vmax[unit * kD + ch] = m;
+}
+
+// Slab blockIdx.x of (b = blockIdx.z, h = blockIdx.y).
+template <bool kNormRope>
+__global__ void __launch_bounds__(kStatsThreads) stats_kernel(const PrepParams p) {
+  __shared__ __align__(16) uint16_t ks[kTile * kD];  // [row][channel] BF16
+  __shared__ VRed vred[kStatsThreads / 32];
+  stats_slab<kNormRope>(p, blockIdx.x, blockIdx.y, blockIdx.z, ks, vred);
 }
 
 // --------------------------------------------------------------- finalize ----
@@ -614,14 +583,18 @@ __global__ void __launch_bounds__(256, 2) quantize_kernel(const PrepParams p) {
 // as the three-kernel path.  Every stage's global writes are read by other threads of
 // the block only after a block barrier.
 template <bool kNormRope>
-__global__ void __launch_bounds__(256, 1) prep_small_kernel(const PrepParams p) {
+__global__ void __launch_bounds__(kStatsThreads, 1) prep_small_kernel(const PrepParams p) {
   __shared__ float red[8];
   __shared__ float gmax[4];
-  __shared__ __align__(16) uint8_t vt[kD * kTile];
+  // the statistics' staged K and V maxima, then (after a barrier) the V transpose tile
+  __shared__ __align__(16) uint8_t scratch[kTile * kD * 2 + sizeof(VRed) * (kStatsThreads / 32)];
+  uint16_t* ks = reinterpret_cast<uint16_t*>(scratch);
+  VRed* vred = reinterpret_cast<VRed*>(scratch + kTile * kD * 2);
+  uint8_t* vt = scratch;
   const int64_t bh = blockIdx.x;
   if (bh == 0 && threadIdx.x == 0) clear_status(p);
   if (kNormRope) {
-    // Q rows transformed into the Q-word area (half-warp = one row), K rows by stats_unit
+    // Q rows transformed into the Q-word area (half-warp = one row), K rows by stats_slab
     const int c16 = threadIdx.x & 15;
     float g[8];
     load_gamma8(p.gamma_q, c16, g);
@@ -631,9 +604,10 @@ __global__ void __launch_bounds__(256, 1) prep_small_kernel(const PrepParams p) 
           norm_rope_row(ldg16(qp + t * p.qst), g, p.cos_q + t * (kD / 2) + 4 * c16, p.sin_q + t * (kD / 2) + 4 * c16,
                         p.eps, half_warp_mask());
   }
-  for (int64_t c = threadIdx.x >> 4; c < p.nchunk; c += blockDim.x >> 4)
-    stats_unit<kNormRope>(p, bh * p.nchunk + c, (int)(threadIdx.x & 15));
-  __syncthreads();
+  for (int64_t slab = 0; slab < p.Tkv_pad / kTile; ++slab) {
+    stats_slab<kNormRope>(p, slab, bh % p.H, bh / p.H, ks, vred);
+    __syncthreads();  // ks and vred are rewritten by the next slab
+  }
   if (threadIdx.x < kD) finalize_channel(p, bh, threadIdx.x);
   __syncthreads();
   const int64_t slabs = (p.Tq_pad > p.Tkv_pad ? p.Tq_pad : p.Tkv_pad) / kTile;
