@@ -97,8 +97,8 @@ h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_v
     return H3ATTN_ERR_WORKSPACE;
 
   const int g = heads_per_group, ngroups = (H + g - 1) / g;
-  Slot sl;
-  make_slot(B, Tq, Tkv, g, &sl);
+  Slot sl{};
+  if (!make_slot(B, Tq, Tkv, g, &sl)) return H3ATTN_ERR_INVALID_ARG;
   char* base = static_cast<char*>(dev_buf);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
@@ -173,8 +173,8 @@ h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int
                                                int heads_per_group, void* stream) {
   if (h3attn_forward_host_bytes(B, Tq, Tkv, H, D, heads_per_group) == 0) return H3ATTN_ERR_INVALID_ARG;
   if (dev_buf == nullptr || reinterpret_cast<uintptr_t>(dev_buf) % 1024 != 0) return H3ATTN_ERR_WORKSPACE;
-  Slot sl;
-  make_slot(B, Tq, Tkv, heads_per_group, &sl);
+  Slot sl{};
+  if (!make_slot(B, Tq, Tkv, heads_per_group, &sl)) return H3ATTN_ERR_INVALID_ARG;
   h3attn_status first = H3ATTN_OK;
   const int used = (H + heads_per_group - 1) / heads_per_group >= 2 ? 2 : 1;  // an unused slot holds no status
   for (int slot = 0; slot < used; ++slot) {
