@@ -206,6 +206,15 @@ def traffic_record(w):
     return rec
 
 
+def launches_per_step(w) -> int:
+    """Kernels one forward launches: the preparation (one kernel for sequences of at most 4
+    slabs of 128 tokens, else statistics + ordered reduction + quantize, plus the Q transform
+    with the norm + RoPE) and the attention."""
+    slabs = max(-(-w.Tq // 128), -(-w.Tkv // 128))
+    prep = 1 if slabs <= 4 else 3 + (1 if w.norm_rope else 0)
+    return prep + 1
+
+
 def max_over_ranks(dist, val: float, device) -> float:
     """The slowest rank's value (all ranks take part; dist None = single process)."""
     if dist is None:
@@ -420,7 +429,8 @@ def run_ours(args, w):
     line = {"metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic", "config": config_of(w, world),
-            "clocks": clk, "gpu_launches": 4 * K, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu}
+            "clocks": clk, "gpu_launches": launches_per_step(w) * K, "roofline": roofline, "e2e": e2e,
+            "cpu_baseline": cpu}
     if norm_rope is not None:
         line["norm_rope"] = norm_rope
         line["e2e_note"] = "the host-buffer pipeline has no norm + RoPE variant; e2e is measured on the plain workloads"
