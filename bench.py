@@ -415,6 +415,10 @@ def run_ours(args, w):
                 # stats reads K, V (4 B); quantize reads Q, K, V (2 + 4 B) and writes the Q, K words
                 # (2 + 2 B, INT8 values held as BF16) and v8 (1 B)
                 "quantize_gbs": (11 * w.Tkv + 4 * w.Tq) * w.B * w.H * w.D / (quant_avg * 1e-3) / 1e9}
+    if "hbm_gbs" in peaks:
+        # the preparation kernels are HBM-bound: their algorithmic bytes against the measured copy rate
+        roofline["quantize_frac_of_hbm"] = roofline["quantize_gbs"] / peaks["hbm_gbs"]
+        roofline["hbm_peak_gbs"] = peaks["hbm_gbs"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
