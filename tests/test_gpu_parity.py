@@ -401,3 +401,42 @@ def test_random_shapes_against_the_oracle():
         ws, out, out4 = run_forward(w, d)
         check_quantized(ws, z, w)
         compare_out(bits(out4), oracle.attend_all(z, w.scale, EPOCH), w.name)
+
+
+def test_concurrent_host_threads():
+    """Four host threads call the library at once (ctypes releases the GIL), each on its
+    own stream and workspace; every output equals the single-threaded result."""
+    import threading
+    w = synth.Workload("threads", 1, 600, 600, 2, 128, "rmsnorm", 8201)
+    x = synth.make_inputs(w)
+    d = upload(x, w)
+    ws0 = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    ref = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    h3.h3attn_forward(d["q"], d["k"], d["v"], w.scale, ref, ws0)
+    assert h3.h3attn_check_status(ws0) == h3.OK
+    n = 4
+    streams = [torch.cuda.Stream() for _ in range(n)]
+    wss = [h3.new_workspace(w.B, w.Tq, w.Tkv, w.H) for _ in range(n)]
+    outs = [torch.zeros_like(ref) for _ in range(n)]
+    errors = []
+    torch.cuda.synchronize()
+
+    def worker(i):
+        try:
+            torch.cuda.set_device(0)
+            for _ in range(10):
+                h3.h3attn_forward(d["q"], d["k"], d["v"], w.scale, outs[i], wss[i], stream=streams[i])
+            if h3.h3attn_check_status(wss[i], streams[i]) != h3.OK:
+                errors.append(f"thread {i}: device status")
+        except Exception as e:  # reported below, in the test's own thread
+            errors.append(f"thread {i}: {e!r}")
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(n)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    torch.cuda.synchronize()
+    for o in outs:
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
