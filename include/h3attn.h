@@ -30,7 +30,7 @@
  *     streams and eight events per call and releases them before it returns, and
  *     h3attn_forward_static uses its own static device array.  Other than that
  *     array, the library keeps no state between calls beyond per-device caches of
- *     kernel attributes and the array's address.
+ *     kernel attributes.
  *   - Element strides are in BF16 elements; the channel (d) stride is 1.
  *     Base pointers must be 16-byte aligned and strides multiples of 8
  *     elements (16-byte vector loads); the workspace must be 256-byte aligned.
@@ -38,7 +38,11 @@
  *     stream) and runs asynchronously.  Argument errors are returned
  *     synchronously and nothing is enqueued.  Errors found on the device (a
  *     bounded wait that expired) are recorded in the workspace's status word
- *     and returned by h3attn_check_status.
+ *     and returned by h3attn_check_status.  The status word is sticky: the
+ *     first failure of any call made on a workspace stays recorded, through
+ *     later calls on the same workspace, until h3attn_check_status reads and
+ *     clears it.  (The quantize pass initialises the status block only on a
+ *     workspace that does not hold its 64-bit marker yet, i.e. a new one.)
  *   - Inputs are assumed finite; NaN or Inf inputs give undefined output.
  *   - Output must not overlap the inputs or the workspace.
  */
@@ -83,7 +87,7 @@ typedef struct {
 
 /* Workspace fields, in the order h3attn_workspace_layout reports their byte offsets. */
 enum {
-  H3ATTN_WS_STATUS = 0, /* int32 status word (+ detail words), 256 bytes */
+  H3ATTN_WS_STATUS = 0, /* status block, 256 bytes: int32 code, detail, block, 64-bit marker */
   H3ATTN_WS_Q8,         /* INT8 Q words held as BF16 values (exact), [B, H, Tq_pad, 128];
                            Tq_pad = ceil(Tq/128)*128, rows >= Tq are 0 */
   H3ATTN_WS_K8,         /* INT8 K words held as BF16 values, [B, H, Tkv_pad, 128];
@@ -109,7 +113,8 @@ h3attn_status h3attn_workspace_layout(int B, int Tq, int Tkv, int H, int D,
 /* K smoothing, Q/K INT8 and V FP8 quantization ("H3 Performance Roadmap", the
  * Sage2 decomposition: K smoothing, Q/K INT8 quantization, V transpose and FP8
  * quantization).  Reads q (Tq tokens) and k, v (Tkv tokens); writes every
- * field of the workspace and clears its status word.  Three kernels (per-chunk
+ * field of the workspace (the status block only when it is new, see the
+ * conventions above).  Three kernels (per-chunk
  * statistics, their ordered reduction, one quantize pass), or one kernel doing
  * all three per (b, h) when max(Tq, Tkv) is at most 512 tokens; both give the
  * same words. */
@@ -139,7 +144,8 @@ h3attn_status h3attn_forward_ex(const h3attn_bf16_view* q, const h3attn_bf16_vie
                                 void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns the device status recorded in the workspace
- * (H3ATTN_OK or H3ATTN_ERR_TIMEOUT) and clears it.  ws must be at least 256 bytes. */
+ * (H3ATTN_OK or H3ATTN_ERR_TIMEOUT: the first failure of any call on this workspace
+ * since the last check) and clears it.  ws must be at least 256 bytes. */
 h3attn_status h3attn_check_status(void* ws, void* stream);
 
 /* Parity export: the exact INT32 QK^T tile of (b, h, Q tile qt, key tile kt) as
@@ -182,9 +188,23 @@ h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_v
                                   void* dev_buf, size_t dev_bytes, void* stream);
 
 /* h3attn_check_status for the workspaces inside an h3attn_forward_host buffer: the
- * first non-OK status of the slots the call used (each is read and cleared). */
+ * first non-OK status of the slots the calls used (each is read and cleared).  The
+ * status words are sticky, so a timeout in any head group of any call since the last
+ * check is reported, not only one in the last two groups. */
 h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int Tkv, int H, int D,
                                                int heads_per_group, void* stream);
+
+/* Failure-path test hook of the host pipeline: h3attn_forward_host with the attention of
+ * head group fail_group (0 <= fail_group < ceil(H / heads_per_group)) launched through
+ * h3attn_debug_attend_timeout (waits bounded by wait_limit_ns, 1 ms to 2 s, the O-ready
+ * arrivals withheld), every other group as usual.  h3attn_forward_host_check_status then
+ * reports H3ATTN_ERR_TIMEOUT, whichever group failed; the other groups' output heads are
+ * those of h3attn_forward_host.  No fault, trap or unbounded wait is involved. */
+h3attn_status h3attn_debug_forward_host_timeout(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                                const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H,
+                                                int D, float softmax_scale, const h3attn_bf16_out* out,
+                                                int heads_per_group, void* dev_buf, size_t dev_bytes,
+                                                int fail_group, uint64_t wait_limit_ns, void* stream);
 
 /* Failure-path test hook: h3attn_attend with every barrier wait bounded by
  * wait_limit_ns (1 ms to 2 s) and the correction warpgroup's "O ready" arrivals
@@ -225,21 +245,40 @@ h3attn_status h3attn_debug_attend_trace(const void* ws, size_t ws_bytes, int B, 
 /* Size of the device array behind h3attn_forward_static (64 MiB). */
 #define H3ATTN_STATIC_WS_BYTES (64u << 20)
 
+/* H3ATTN_STATIC_WS_BYTES as compiled into the loaded library. */
+size_t h3attn_static_workspace_bytes(void);
+
 /* Forward pass (quantize + attend, Tq and Tkv as in h3attn_forward_ex) for callers that
  * cannot allocate device memory: a host that owns the device allocator and offers this
  * library no way to request memory, or a runtime that forbids allocation after start-up.
  * The pages have no counterpart; it is an interface addition of this library.
  * Takes the inputs and the output only. The workspace is a file-scope device array of
  * H3ATTN_STATIC_WS_BYTES that every GPU loading the library holds until exit; shapes
- * whose h3attn_workspace_bytes exceeds it return H3ATTN_ERR_WORKSPACE. The first call
- * on a device (with that device current) looks up the array's address; make that first
- * call before any stream capture. Calls no cudaMalloc or cudaFree. All calls share the
- * array, which keeps the last call's contents, so calls whose GPU work overlaps race on
- * it; the caller must order them. Device-side wait timeouts are recorded in the array's
- * status word, which this interface does not expose. */
+ * whose h3attn_workspace_bytes exceeds it return H3ATTN_ERR_WORKSPACE before anything is
+ * enqueued. Every call looks up the array's device address for the current device and
+ * context (cudaGetSymbolAddress, a host-side query); the first call on a device also makes
+ * the runtime load the library's device code there, so make that first call before any
+ * stream capture. Calls no cudaMalloc or cudaFree. All calls share the array, which keeps
+ * the last call's contents, so calls whose GPU work overlaps race on it; the caller must
+ * order them. Device-side wait timeouts are recorded in the array's sticky status word:
+ * read it with h3attn_static_check_status. */
 h3attn_status h3attn_forward_static(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
                                     const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
                                     float softmax_scale, const h3attn_bf16_out* out, void* stream);
+
+/* h3attn_check_status on the static array of h3attn_forward_static (current device):
+ * synchronises `stream`, returns the first device-side failure of any static call since
+ * the last check (H3ATTN_OK or H3ATTN_ERR_TIMEOUT) and clears it.  Like the entry point
+ * it serves, it allocates nothing. */
+h3attn_status h3attn_static_check_status(void* stream);
+
+/* Failure-path test hook on the static array: h3attn_debug_attend_timeout run on the
+ * workspace that the last h3attn_forward_static call of the same sizes filled.  Sizes
+ * that do not fit the array return H3ATTN_ERR_WORKSPACE; h3attn_static_check_status then
+ * reports H3ATTN_ERR_TIMEOUT. */
+h3attn_status h3attn_debug_static_attend_timeout(int B, int Tq, int Tkv, int H, int D, float softmax_scale,
+                                                 const h3attn_bf16_out* out, uint64_t wait_limit_ns,
+                                                 void* stream);
 
 /* ---- Q/K RMSNorm + RoPE before the attention ("H3 Performance Roadmap", Component 2
  * execution order, item 1: Q/K normalization and RoPE where the attention consumes Q

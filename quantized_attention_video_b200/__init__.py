@@ -70,6 +70,12 @@ def lib() -> ctypes.CDLL:
         L.h3attn_forward_ex.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, P, S, P]
         L.h3attn_forward_static.restype = I
         L.h3attn_forward_static.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, P]
+        L.h3attn_static_workspace_bytes.restype = S
+        L.h3attn_static_workspace_bytes.argtypes = []
+        L.h3attn_static_check_status.restype = I
+        L.h3attn_static_check_status.argtypes = [P]
+        L.h3attn_debug_static_attend_timeout.restype = I
+        L.h3attn_debug_static_attend_timeout.argtypes = [I] * 5 + [F, VP, ctypes.c_uint64, P]
         L.h3attn_check_status.restype = I
         L.h3attn_check_status.argtypes = [P, P]
         L.h3attn_debug_qk_scores.restype = I
@@ -84,6 +90,9 @@ def lib() -> ctypes.CDLL:
         L.h3attn_forward_host.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, I, P, S, P]
         L.h3attn_forward_host_check_status.restype = I
         L.h3attn_forward_host_check_status.argtypes = [P] + [I] * 6 + [P]
+        L.h3attn_debug_forward_host_timeout.restype = I
+        L.h3attn_debug_forward_host_timeout.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, I, P, S, I,
+                                                                                  ctypes.c_uint64, P]
         NP = ctypes.POINTER(_NormRope)
         L.h3attn_quantize_qkv_norm_rope.restype = I
         L.h3attn_quantize_qkv_norm_rope.argtypes = [VP, VP, VP] + [I] * 5 + [NP, P, S, P]
@@ -268,7 +277,39 @@ def h3attn_forward_host_check_status(dev_buf, B: int, Tq: int, Tkv: int, H: int,
                                                   _stream(stream))
 
 
-STATIC_WS_BYTES = 64 << 20
+def h3attn_debug_forward_host_timeout(q, k, v, softmax_scale: float, out, dev_buf, heads_per_group: int,
+                                      fail_group: int, wait_limit_ns: int, stream=None):
+    """h3attn_forward_host with head group fail_group's waits bounded and withheld (test hook)."""
+    B, Tq, H, D = q.shape
+    Tkv = k.shape[1]
+    wp, wb = _ptr_bytes(dev_buf)
+    vq, vk, vv, vo = _view(q), _view(k), _view(v), _view(out)
+    _check(lib().h3attn_debug_forward_host_timeout(ctypes.byref(vq), ctypes.byref(vk), ctypes.byref(vv), B, Tq, Tkv,
+                                                   H, D, softmax_scale, ctypes.byref(vo), heads_per_group, wp, wb,
+                                                   fail_group, int(wait_limit_ns), _stream(stream)),
+           "h3attn_debug_forward_host_timeout")
+
+
+STATIC_WS_BYTES = 64 << 20  # H3ATTN_STATIC_WS_BYTES (the tests compare it with the loaded library's value)
+
+
+def h3attn_static_workspace_bytes() -> int:
+    """Size of the library's static device array (read from the loaded library)."""
+    return lib().h3attn_static_workspace_bytes()
+
+
+def h3attn_static_check_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the static array's sticky status word."""
+    return lib().h3attn_static_check_status(_stream(stream))
+
+
+def h3attn_debug_static_attend_timeout(B: int, Tq: int, Tkv: int, H: int, softmax_scale: float, out,
+                                       wait_limit_ns: int, stream=None, D: int = HEAD_DIM):
+    """The timeout test hook run on the static array (after an h3attn_forward_static of the same sizes)."""
+    vo = _view(out)
+    _check(lib().h3attn_debug_static_attend_timeout(B, Tq, Tkv, H, D, softmax_scale, ctypes.byref(vo),
+                                                    int(wait_limit_ns), _stream(stream)),
+           "h3attn_debug_static_attend_timeout")
 
 
 def h3attn_forward_static(q, k, v, softmax_scale: float, out, stream=None):
@@ -324,7 +365,8 @@ def h3attn_debug_attend_timeout(ws, B: int, Tq: int, Tkv: int, H: int, softmax_s
 
 
 def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:
-    """Typed views of the workspace fields (for parity checks; q8/k8 are INT8 copies)."""
+    """Views of the workspace fields as stored (no copies, no conversions): q8/k8 are the
+    INT8 words held as BF16 values (torch.bfloat16; compare their bit patterns)."""
     import torch
     off = h3attn_workspace_layout(B, Tq, Tkv, H)
     Tqp, Tkp = -(-Tq // TILE) * TILE, -(-Tkv // TILE) * TILE
@@ -334,10 +376,9 @@ def workspace_views(ws, B: int, Tq: int, Tkv: int, H: int) -> dict:
         return ws[off[name]:off[name] + nb].view(dtype).view(shape)
 
     BH = B * H
-    # the INT8 Q/K words are stored as BF16 values (exact); inspect them as INT8
     return dict(
-        q8=sl("q8", BH * Tqp * 128, torch.bfloat16, (B, H, Tqp, 128)).to(torch.int8),
-        k8=sl("k8", BH * Tkp * 128, torch.bfloat16, (B, H, Tkp, 128)).to(torch.int8),
+        q8=sl("q8", BH * Tqp * 128, torch.bfloat16, (B, H, Tqp, 128)),
+        k8=sl("k8", BH * Tkp * 128, torch.bfloat16, (B, H, Tkp, 128)),
         v8t=sl("v8t", BH * 128 * Tkp, torch.uint8, (B, H, 128, Tkp)),
         sq=sl("sq", BH * (Tqp // Q_GROUP), torch.float32, (B, H, Tqp // Q_GROUP)),
         sk=sl("sk", BH * (Tkp // K_GROUP), torch.float32, (B, H, Tkp // K_GROUP)),

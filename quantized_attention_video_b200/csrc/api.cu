@@ -195,7 +195,11 @@ h3attn_status h3attn_check_status(void* ws, void* stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return H3ATTN_ERR_CUDA;
   int code = 0;
   if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return H3ATTN_ERR_CUDA;
-  if (cudaMemset(ws, 0, sizeof(DevStatus)) != cudaSuccess) return H3ATTN_ERR_CUDA;
+  // clear the code, detail and block words and leave the block initialised (marker
+  // set), so that the next quantize pass keeps, rather than re-initialises, whatever a
+  // later call records
+  const uint32_t fresh[5] = {0u, 0u, 0u, kStatusMarker0, kStatusMarker1};
+  if (cudaMemcpy(ws, fresh, sizeof(fresh), cudaMemcpyHostToDevice) != cudaSuccess) return H3ATTN_ERR_CUDA;
   if (code < 0 || code > H3ATTN_ERR_TIMEOUT) return H3ATTN_ERR_CUDA;
   return static_cast<h3attn_status>(code);
 }

@@ -77,10 +77,17 @@ size_t h3attn_forward_host_bytes(int B, int Tq, int Tkv, int H, int D, int heads
   return 2 * s.bytes;
 }
 
-h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_view* k, const h3attn_bf16_view* v,
-                                  int B, int Tq, int Tkv, int H, int D, float softmax_scale,
-                                  const h3attn_bf16_out* out, int heads_per_group, void* dev_buf,
-                                  size_t dev_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The pipeline of h3attn_forward_host.  fail_group >= 0 (test hook): that group's
+// attention runs through h3attn_debug_attend_timeout with waits bounded by
+// wait_limit_ns, so it records a device-side timeout in its slot's status word.
+h3attn_status forward_host_impl(const h3attn_bf16_view* q, const h3attn_bf16_view* k, const h3attn_bf16_view* v,
+                                int B, int Tq, int Tkv, int H, int D, float softmax_scale,
+                                const h3attn_bf16_out* out, int heads_per_group, void* dev_buf, size_t dev_bytes,
+                                void* stream, int fail_group, uint64_t wait_limit_ns) {
   const size_t need = h3attn_forward_host_bytes(B, Tq, Tkv, H, D, heads_per_group);
   if (need == 0) return D != kD ? H3ATTN_ERR_UNSUPPORTED : H3ATTN_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return H3ATTN_ERR_INVALID_ARG;
@@ -152,7 +159,15 @@ h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_v
     const h3attn_bf16_view dk = {sb + sl.k, (int64_t)Tkv * tk, tk, kD};
     const h3attn_bf16_view dv = {sb + sl.v, (int64_t)Tkv * tk, tk, kD};
     const h3attn_bf16_out dout = {sb + sl.o, (int64_t)Tq * tq, tq, kD};
-    result = h3attn_forward_ex(&dq, &dk, &dv, B, Tq, Tkv, gn, D, softmax_scale, &dout, sb + sl.ws, sl.ws_bytes, cs);
+    if (gi == fail_group) {
+      result = h3attn_quantize_qkv(&dq, &dk, &dv, B, Tq, Tkv, gn, D, sb + sl.ws, sl.ws_bytes, cs);
+      if (result == H3ATTN_OK)
+        result = h3attn_debug_attend_timeout(sb + sl.ws, sl.ws_bytes, B, Tq, Tkv, gn, D, softmax_scale, &dout,
+                                             wait_limit_ns, cs);
+    } else {
+      result = h3attn_forward_ex(&dq, &dk, &dv, B, Tq, Tkv, gn, D, softmax_scale, &dout, sb + sl.ws, sl.ws_bytes,
+                                 cs);
+    }
     if (result != H3ATTN_OK) break;
     ok = cudaEventRecord(ev_comp[slot], cs) == cudaSuccess;
     // download
@@ -167,6 +182,29 @@ h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_v
   release();
   if (result != H3ATTN_OK) return result;
   return ok && joined ? H3ATTN_OK : H3ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_view* k, const h3attn_bf16_view* v,
+                                  int B, int Tq, int Tkv, int H, int D, float softmax_scale,
+                                  const h3attn_bf16_out* out, int heads_per_group, void* dev_buf,
+                                  size_t dev_bytes, void* stream) {
+  return forward_host_impl(q, k, v, B, Tq, Tkv, H, D, softmax_scale, out, heads_per_group, dev_buf, dev_bytes,
+                           stream, -1, 0);
+}
+
+h3attn_status h3attn_debug_forward_host_timeout(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
+                                                const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
+                                                float softmax_scale, const h3attn_bf16_out* out,
+                                                int heads_per_group, void* dev_buf, size_t dev_bytes,
+                                                int fail_group, uint64_t wait_limit_ns, void* stream) {
+  if (heads_per_group < 1 || fail_group < 0 || fail_group >= (H + heads_per_group - 1) / heads_per_group)
+    return H3ATTN_ERR_INVALID_ARG;
+  return forward_host_impl(q, k, v, B, Tq, Tkv, H, D, softmax_scale, out, heads_per_group, dev_buf, dev_bytes,
+                           stream, fail_group, wait_limit_ns);
 }
 
 h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int Tkv, int H, int D,

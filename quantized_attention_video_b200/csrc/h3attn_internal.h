@@ -68,13 +68,19 @@ inline h3attn_status check_strides(const void* data, int64_t sb, int64_t st, int
   return H3ATTN_OK;
 }
 
-// Device-side status words at the start of the workspace.
+// Device-side status words at the start of the workspace.  The status is sticky: a
+// quantize pass initialises the block only when its two marker words are missing (a
+// new workspace), and h3attn_check_status clears the code but keeps the marker, so a
+// failure recorded by any call stays until h3attn_check_status reads and clears it.
+constexpr uint32_t kStatusMarker0 = 0x68336174u, kStatusMarker1 = 0x74737453u;
 struct DevStatus {
   int code;    // h3attn_status of the first failure, 0 if none
   int detail;  // which wait expired (kernel-defined id)
   int block;   // linear block index that recorded it
-  int pad[61];
+  uint32_t marker[2];  // kStatusMarker0, kStatusMarker1 once initialised
+  int pad[59];
 };
+static_assert(sizeof(DevStatus) == 256, "status block size");
 
 // Kernel launchers (defined in quantize.cu / attention.cu).
 // nr != nullptr: Q and K rows pass through the RMSNorm + RoPE transform as they are loaded.

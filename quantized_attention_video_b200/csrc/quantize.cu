@@ -290,11 +290,18 @@ __device__ __forceinline__ void finalize_channel(const PrepParams& p, int64_t bh
   vp[0] = m;
 }
 
-// Clears the workspace status word, so each quantize call starts clean.
-__device__ __forceinline__ void clear_status(const PrepParams& p) {
-  p.status->code = 0;
-  p.status->detail = 0;
-  p.status->block = 0;
+// Initialises the workspace status block of a new workspace (marker words absent).  An
+// initialised block is left alone, so a failure recorded by an earlier call on this
+// workspace survives until h3attn_check_status reads and clears it.
+__device__ __forceinline__ void init_status(const PrepParams& p) {
+  DevStatus* st = p.status;
+  if (st->marker[0] != kStatusMarker0 || st->marker[1] != kStatusMarker1) {
+    st->code = 0;
+    st->detail = 0;
+    st->block = 0;
+    st->marker[0] = kStatusMarker0;
+    st->marker[1] = kStatusMarker1;
+  }
 }
 
 // Block (b*H + h = blockIdx.x, channels [32*blockIdx.y, 32*blockIdx.y + 32)); lane =
@@ -313,7 +320,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const PrepParams 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = blockIdx.x;
   const int c = blockIdx.y * 32 + lane;
-  if (bh == 0 && blockIdx.y == 0 && tid == 0) clear_status(p);
+  if (bh == 0 && blockIdx.y == 0 && tid == 0) init_status(p);
   const double* kp = p.ksum + bh * p.nchunk * kD + c;
   float* vp = p.vmax + bh * p.nchunk * kD + c;
   const int64_t npass = (p.nchunk + kFinRows - 1) / kFinRows;
@@ -592,7 +599,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1) prep_small_kernel(const Prep
   VRed* vred = reinterpret_cast<VRed*>(scratch + kTile * kD * 2);
   uint8_t* vt = scratch;
   const int64_t bh = blockIdx.x;
-  if (bh == 0 && threadIdx.x == 0) clear_status(p);
+  if (bh == 0 && threadIdx.x == 0) init_status(p);
   if (kNormRope) {
     // Q rows transformed into the Q-word area (half-warp = one row), K rows by stats_slab
     const int c16 = threadIdx.x & 15;

@@ -91,3 +91,53 @@ def test_timeout_hook_rejects_out_of_range_limits():
     for bad in (0, 999_999, 3_000_000_000):
         with pytest.raises(h3.H3AttnError):
             h3.h3attn_debug_attend_timeout(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, bad)
+
+
+def test_status_is_sticky_across_later_calls():
+    """A timeout recorded by one call survives later calls on the same workspace (their
+    preparation does not clear it) until h3attn_check_status reads it ("Phase 2B Aligned
+    Numerical Prototype", Synchronization And Safety: a failure must not be lost)."""
+    w, q, k, v = _inputs("fixed_q128_kv192")
+    ws = h3.new_workspace(w.B, w.Tq, w.Tkv, w.H)
+    out = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    h3.h3attn_forward_ex(q, k, v, w.scale, out, ws)
+    assert h3.h3attn_check_status(ws) == h3.OK
+    h3.h3attn_debug_attend_timeout(ws, w.B, w.Tq, w.Tkv, w.H, w.scale, out, LIMIT_NS)
+    for _ in range(3):  # later, successful calls on the same workspace
+        h3.h3attn_forward_ex(q, k, v, w.scale, out, ws)
+    assert h3.h3attn_check_status(ws) == h3.ERR_TIMEOUT
+    assert h3.h3attn_check_status(ws) == h3.OK
+
+
+@pytest.mark.parametrize("fail_group", [0, 1, 2])
+def test_host_pipeline_reports_an_early_group_timeout(fail_group):
+    """h3attn_forward_host over 4 head groups (two device slots reused in turn) with the
+    waits of one early group withheld: h3attn_forward_host_check_status reports the
+    timeout although two later groups reused that group's slot; the heads of the other
+    groups are those of the normal pipeline."""
+    w = synth.WORKLOADS["selfattn_h8_t4096"]
+    x = synth.make_inputs(w)
+    host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    q, k, v = host(x["q"]), host(x["k"]), host(x["v"])
+    g = 2  # 8 heads -> 4 groups
+    buf = h3.new_host_buffer(w.B, w.Tq, w.Tkv, w.H, g)
+    ref = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16).pin_memory()
+    h3.h3attn_forward_host(q, k, v, w.scale, ref, buf, g)
+    assert h3.h3attn_forward_host_check_status(buf, w.B, w.Tq, w.Tkv, w.H, g) == h3.OK
+    out = torch.zeros_like(ref).pin_memory()
+    h3.h3attn_debug_forward_host_timeout(q, k, v, w.scale, out, buf, g, fail_group, LIMIT_NS)
+    assert h3.h3attn_forward_host_check_status(buf, w.B, w.Tq, w.Tkv, w.H, g) == h3.ERR_TIMEOUT
+    assert h3.h3attn_forward_host_check_status(buf, w.B, w.Tq, w.Tkv, w.H, g) == h3.OK
+    others = [h for h in range(w.H) if h // g != fail_group]
+    assert torch.equal(out[:, :, others].view(torch.int16), ref[:, :, others].view(torch.int16))
+
+
+def test_host_timeout_hook_rejects_a_group_out_of_range():
+    w = synth.WORKLOADS["fixed_q128_kv192"]
+    x = synth.make_inputs(w)
+    host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    q, k, v = host(x["q"]), host(x["k"]), host(x["v"])
+    buf = h3.new_host_buffer(w.B, w.Tq, w.Tkv, w.H, 1)
+    out = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16).pin_memory()
+    with pytest.raises(h3.H3AttnError):
+        h3.h3attn_debug_forward_host_timeout(q, k, v, w.scale, out, buf, 1, 1, LIMIT_NS)

@@ -65,13 +65,23 @@ def f32_bits(a: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.float32).view(np.int32)
 
 
+def int8_as_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """The exact BF16 encoding of integer words in [-127, 127] (the form the workspace
+    stores them in): the top half of their FP32 encoding, whose low half is zero."""
+    f = np.ascontiguousarray(a, dtype=np.int8).astype(np.float32).view(np.uint32)
+    assert not (f & 0xFFFF).any()
+    return (f >> 16).astype(np.uint16)
+
+
 def check_quantized(ws, z, w):
     B, Tq, Tkv, H = w.B, w.Tq, w.Tkv, w.H
     v = h3.workspace_views(ws, B, Tq, Tkv, H)
+    # the stored bit patterns of the Q/K words against the exact encoding of the
+    # oracle's integers (no conversion of the GPU's words), padding +0 exactly
     q8, k8, v8t = bits(v["q8"]), bits(v["k8"]), bits(v["v8t"])
-    assert np.array_equal(q8[:, :, :Tq], z["q8"]), "q8"
+    assert np.array_equal(q8[:, :, :Tq], int8_as_bf16_bits(z["q8"])), "q8"
     assert not q8[:, :, Tq:].any()
-    assert np.array_equal(k8[:, :, :Tkv], z["k8"]), "k8"
+    assert np.array_equal(k8[:, :, :Tkv], int8_as_bf16_bits(z["k8"])), "k8"
     assert not k8[:, :, Tkv:].any()
     assert np.array_equal(v8t[:, :, :, :Tkv].transpose(0, 1, 3, 2), z["v8"]), "v8"
     assert not v8t[:, :, :, Tkv:].any()
@@ -96,15 +106,23 @@ def compare_out(got: np.ndarray, ref: np.ndarray, what: str):
     return err.max(), rel
 
 
-def sample_rows(w: synth.Workload, tiles_per_head: int, seed: int):
-    """(b, h, i) rows: the first and last (ragged) Q tile of every head plus random tiles."""
+def sample_tiles(ntile: int, n_random: int, rng) -> list:
+    """Q tiles checked for one (b, h): the first two and the last two (the ragged tail
+    among them) plus n_random distinct seeded interior tiles."""
+    fixed = {t for t in (0, 1, ntile - 2, ntile - 1) if 0 <= t < ntile}
+    interior = [t for t in range(ntile) if t not in fixed]
+    picked = rng.choice(interior, size=min(n_random, len(interior)), replace=False) if interior else []
+    return sorted(fixed | {int(t) for t in picked})
+
+
+def sample_rows(w: synth.Workload, n_random: int, seed: int):
+    """(b, h, i) rows of sample_tiles for every batch item and head."""
     rng = np.random.default_rng(seed)
     ntile = -(-w.Tq // 128)
     rows = []
     for b in range(w.B):
         for h in range(w.H):
-            tiles = {0, ntile - 1} | set(rng.integers(0, ntile, size=tiles_per_head).tolist())
-            for t in sorted(tiles):
+            for t in sample_tiles(ntile, n_random, rng):
                 for i in range(t * 128, min(w.Tq, t * 128 + 128)):
                     rows.append((b, h, i))
     return np.array(rows, dtype=np.int32)
@@ -122,8 +140,17 @@ def run_forward(w, d):
 
 
 # ---------------------------------------------------------------- configs ----
+# Output rows compared with the oracle: every row of the first two workloads; for the
+# others, every (b, h) with its first two and last two Q tiles plus 8 seeded interior
+# ones (sample_tiles):
+#   ragged_h16_t9453     16 heads x (11 x 128 + 109) rows        = 24,272 rows
+#   h3_t37810_h32        32 heads x (11 x 128 + 50) rows         = 46,656 rows
+#   h3_packed_b2_t37810  2 batch items x 32 heads x 1,458 rows   = 93,312 rows
+#   h3_t74000_h32        32 heads x (11 x 128 + 16) rows         = 45,568 rows
 FULL = ["fixed_q128_kv192", "selfattn_h8_t4096"]
-SAMPLED = {"ragged_h16_t9453": 3, "h3_t37810_h32": 1, "h3_packed_b2_t37810": 0, "h3_t74000_h32": 0}
+SAMPLED = {"ragged_h16_t9453": 8, "h3_t37810_h32": 8, "h3_packed_b2_t37810": 8, "h3_t74000_h32": 8}
+SAMPLED_ROWS = {"ragged_h16_t9453": 24272, "h3_t37810_h32": 46656, "h3_packed_b2_t37810": 93312,
+                "h3_t74000_h32": 45568}
 
 
 @pytest.mark.parametrize("name", FULL + list(SAMPLED))
@@ -140,6 +167,7 @@ def test_workload_parity(name):
         compare_out(got, ref, name)
     else:
         rows = sample_rows(w, SAMPLED[name], seed=w.seed)
+        assert len(rows) == SAMPLED_ROWS[name]
         ref, _, _ = oracle.attend_rows(z, w.scale, EPOCH, rows)
         compare_out(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, name)
     if w.packed:
