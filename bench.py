@@ -22,6 +22,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -153,8 +154,7 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/h3attn_clocks_{os.getpid()}.csv"
+        self.path = os.path.join(tempfile.gettempdir(), f"h3attn_clocks_{os.getpid()}_{index}.csv")
 
     def start(self):
         try:
@@ -399,22 +399,35 @@ def run_ours(args, w):
     pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk_path):
         peaks = json.load(open(pk_path))
-    if "bf16_tflops_sustained" in peaks:
-        peak = 2.0 * peaks["bf16_tflops_sustained"]
-        peak_note = "of measured: 2 x bf16_tflops_sustained (nominal 8-bit/bf16 ratio 2), kernel timed inside a long loop"
+    # The attention kernel runs inside a step of tens of milliseconds, not a seconds-long
+    # loop, so the burst GEMM rate is its peak; the sustained (power-capped) rate is
+    # reported beside it for reference.  8-bit dense = 2 x bf16 dense (nominal ratio).
+    if "bf16_tflops" in peaks:
+        peak = 2.0 * peaks["bf16_tflops"]
+        peak_note = "of measured: 2 x bf16_tflops (burst; nominal 8-bit/bf16 ratio 2)"
     else:
-        peak = 2.0 * 1400.0
-        peak_note = "of fallback: 2 x 1.4 PFLOP/s sustained bf16"
+        peak = 2.0 * 1590.0
+        peak_note = "of fallback: 2 x 1.59 PFLOP/s burst bf16"
     achieved = ops / (attn_avg * 1e-3) / 1e12
     tr = traffic_record(w)
+    bthd = w.B * w.H * w.D
+    # the method's bytes: stats reads K, V (4 B per key); quantize reads Q (2 B), K, V (4 B)
+    # and writes the INT8 Q and K words and the E4M3 V words (1 B each): 13 B per token at
+    # Tq = Tkv.  The Q/K words are stored as BF16 values (2 B each): one extra byte per
+    # word, reported on its own.
+    quant_bytes = (3 * w.Tq + 10 * w.Tkv) * bthd
+    word_overhead = (w.Tq + w.Tkv) * bthd
     roofline = {"bound": "tensor", "kernel": "attn_sm100_kernel", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_note,
                 "algorithmic_ops_per_launch": ops,
                 "traffic": None if tr is None else tr["dram_bytes_per_launch_full"],
                 "quantize_ms": quant_avg, "attention_ms": attn_avg,
-                # stats reads K, V (4 B); quantize reads Q, K, V (2 + 4 B) and writes the Q, K words
-                # (2 + 2 B, INT8 values held as BF16) and v8 (1 B)
-                "quantize_gbs": (11 * w.Tkv + 4 * w.Tq) * w.B * w.H * w.D / (quant_avg * 1e-3) / 1e9}
+                "quantize_algorithmic_bytes": quant_bytes,
+                "quantize_gbs": quant_bytes / (quant_avg * 1e-3) / 1e9,
+                "quantize_word_overhead_bytes": word_overhead}
+    if "bf16_tflops_sustained" in peaks:
+        roofline["peak_sustained"] = 2.0 * peaks["bf16_tflops_sustained"]
+        roofline["frac_of_sustained"] = achieved / roofline["peak_sustained"]
     if "hbm_gbs" in peaks:
         # the preparation kernels are HBM-bound: their algorithmic bytes against the measured copy rate
         roofline["quantize_frac_of_hbm"] = roofline["quantize_gbs"] / peaks["hbm_gbs"]

@@ -336,8 +336,8 @@ def h3attn_debug_qk_scores(ws, B: int, Tq: int, Tkv: int, H: int, b: int, h: int
            "h3attn_debug_qk_scores")
 
 
-TRACE_EVENTS = ("s_ready", "m_pub", "p_done", "qk_issue", "pv_issue", "o_corrected", "k_full", "probs",
-                "pv_done", "s_free", "ld", "max", "p_free", "pv_p", "pv_o", "p_done_last")
+TRACE_EVENTS = ("s_ready", "a_pub", "p_done", "qk_issue", "pv_issue", "o_corrected", "k_full", "probs",
+                "pv_done", "s_free", "ld", "max", "p_free", "pv_p", "pv_o", "turn")
 
 
 def h3attn_debug_attend_trace(ws, B: int, Tq: int, Tkv: int, H: int, softmax_scale: float, out, trace_block: int,

@@ -11,7 +11,8 @@
 //                 S(x) = Q(x) K^T  tcgen05.mma kind::f16 on the INT8 words held
 //                 as BF16 (exact) with FP32 accumulation: every product and
 //                 partial sum is an integer below 2^24, so S equals the INT32
-//                 scores.
+//                 scores.  QK(x, j+1) is issued as soon as softmax x has loaded
+//                 S(x, j), so the next scores are ready before they are needed.
 //        warp 3   PV issuer (one thread):
 //                 O(x) += P(x) V   tcgen05.mma kind::f8f6f4 (E4M3 operands from
 //                 shared memory, F32 accumulate).
@@ -19,18 +20,29 @@
 //                 the two products have their own issuing threads and neither
 //                 waits behind the other's dependencies.
 //   WG1  softmax of Q tile A, WG2 softmax of Q tile B; thread = one Q row, over
-//        every key tile in order.  Each warpgroup owns the whole running max
-//        and row sum of its rows, so the two never wait for each other and
-//        their exp2 phases (bound by the MUFU unit) drift apart instead of
-//        running side by side.
+//        every key tile in order.  Each warpgroup owns the running max and row
+//        sum of its rows.  Their exp2 passes (bound by the MUFU unit) start in
+//        turn A(j) B(j) A(j+1) ...; a warpgroup hands the turn over part-way
+//        through its pass (kTurnHandoverKey), so the end of one pass overlaps the
+//        start of the next and the MUFU unit stays busy through the stalls of
+//        either instruction stream.  Everything else a warpgroup does for a key
+//        tile (score load, row max, probability store) runs while the other
+//        warpgroup has the MUFU unit and holds no MUFU work of its own: the
+//        rescale factor alpha = 2^(m_old - m_new) is the first exp2 of the pass,
+//        and the correction warpgroup reads it instead of computing it.  What
+//        bounds a key tile is the instruction stream of the two softmax
+//        warpgroups on each SM sub-partition, so the pass forms the exp2
+//        arguments next to each exp2 (kFoldArg), converts four probabilities per
+//        instruction (kCvtX4), and the ragged last key tile runs a separate
+//        masked copy after the loop, which keeps the loop's unrolled code (and its
+//        instruction-cache footprint) to one copy.
 //   WG3  O correction of both tiles (rescale by alpha when the running max
 //        moves) and the epilogue (final reciprocal, BF16 store).
 // Tensor memory (512 columns allocated): S(A) [0,128) S(B) [128,256)
 // O(A) [256,384) O(B) [384,512).  The softmax frees S(x) as soon as it has
-// read the scores, so QK of the next key tile runs on the tensor cores while
-// the softmax of this one is still computing.  Its E4M3 probabilities (128 x
-// 128 bytes) go to shared memory in the 128-byte-swizzled K-major layout the
-// PV MMA reads, once PV of the previous key tile has consumed the buffer.
+// read the scores.  Its E4M3 probabilities (128 x 128 bytes) go to shared
+// memory in the 128-byte-swizzled K-major layout the PV MMA reads, once PV of
+// the previous key tile has consumed the buffer.
 //
 // Every wait is bounded: after the limit the waiter records
 // H3ATTN_ERR_TIMEOUT in the workspace status word, raises a CTA-wide abort
@@ -41,6 +53,7 @@
 
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "exp2_poly.h"
 #include "h3attn_internal.h"
@@ -56,6 +69,24 @@ constexpr uint32_t kTileBytes = 128 * 128;          // one 128 x 128-byte swizzl
 constexpr uint32_t kQKTileBytes = 2 * kTileBytes;   // a BF16 128 x 128 tile: two 64-column halves
 __device__ __forceinline__ uint32_t col_s(int x) { return 128u * (uint32_t)x; }        // S(A), S(B)
 __device__ __forceinline__ uint32_t col_o(int x) { return 256u + 128u * (uint32_t)x; } // O(A), O(B)
+// Key (of 128) after which a softmax warpgroup hands the MUFU turn to the other.
+#ifndef H3ATTN_TURN_HANDOVER_KEY
+#define H3ATTN_TURN_HANDOVER_KEY 64
+#endif
+constexpr int kTurnHandoverKey = H3ATTN_TURN_HANDOVER_KEY;
+// 1: the exp2 arguments u = s*f - mq are formed inside the exp2 pass, next to each
+// exp2; 0: in place before the pass (pre_turn).  Either gives the same bits.
+#ifndef H3ATTN_FOLD_ARG
+#define H3ATTN_FOLD_ARG 1
+#endif
+constexpr bool kFoldArg = H3ATTN_FOLD_ARG != 0;
+// 1: four probabilities per conversion instruction (cvt_e4m3x4_half_up) instead of two
+// per instruction and a byte pack.
+#ifndef H3ATTN_CVT_X4
+#define H3ATTN_CVT_X4 1
+#endif
+constexpr bool kCvtX4 = H3ATTN_CVT_X4 != 0;
+static_assert(kTurnHandoverKey >= 0 && kTurnHandoverKey <= 128 && kTurnHandoverKey % 4 == 0, "handover key");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, 128);
 constexpr uint64_t kWaitLimitNs = kDefaultWaitLimitNs;
@@ -71,9 +102,10 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 //   s_full[x]   QK(x,j) done -> softmax x.   QK(x,j+1) needs s_free[x](j).
 //   s_free[x]   softmax x read S(x,j) -> QK issuer.  softmax x reaches the next
 //               arrival only after s_full[x](j+1), which needs this wait.
-//   m_full[x][j%2]  running max of tile j -> correction.  softmax x publishes
-//               m(j+2) only after pv_done[x](j) (P buffer), i.e. after the
-//               correction's o_ready[x](j), which follows its read of m(j).
+//   a_full[x][j%2]  alpha of tile j -> correction.  softmax x publishes alpha
+//               of tile j+2 only after pv_done[x](j) (P buffer free for tile
+//               j+1), i.e. after the correction's o_ready[x](j), which follows
+//               its read of alpha(j).
 //   o_ready[x]  correction -> PV issuer.  The correction waits pv_done[x](j-1)
 //               before arriving for tile j, so phase j-1 has been consumed.
 //   p_full[x]   P(x,j) in shared memory -> PV issuer.  softmax x writes P(x,j+1)
@@ -81,10 +113,12 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 //   pv_done[x]  PV(x,j) done -> softmax x (P buffer free) and correction (O
 //               final up to tile j).  PV(x,j+1) needs p_full[x](j+1) and
 //               o_ready[x](j+1), which both follow these waits.
-//   tok[A]      A's exp2 pass of tile j done -> softmax B (waits phase j).  A's
-//               pass of j+1 needs tok[B](j), which B arrives after this wait.
-//   tok[B]      B's exp2 pass of tile j done -> softmax A (waits phase j before
-//               its pass of j+1).  B's pass of j+1 needs tok[A](j+1), after it.
+//   tok[A]      A's exp2 pass of tile j past the handover key -> softmax B
+//               (waits phase j).  A's pass of j+1 needs tok[B](j), which B
+//               arrives after this wait.
+//   tok[B]      B's exp2 pass of tile j past the handover key -> softmax A
+//               (waits phase j before its pass of j+1).  B's pass of j+1 needs
+//               tok[A](j+1), after it.
 struct __align__(1024) AttnSmem {
   uint8_t q[2][2][kTileBytes];         // [Q tile][half] BF16 Q tiles: key dims [0,64) and [64,128)
   uint8_t k[kStagesK][2][kTileBytes];  // BF16 K tiles, same split
@@ -94,15 +128,15 @@ struct __align__(1024) AttnSmem {
   uint64_t k_full[kStagesK], k_empty[kStagesK];
   uint64_t v_full[kStagesV], v_empty[kStagesV];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], o_ready[2];
-  uint64_t m_full[2][2];
-  uint64_t tok[2];    // [Q tile] softmax x finished its exp2 pass of key tile j (MUFU turn)
+  uint64_t a_full[2][2];
+  uint64_t tok[2];    // [Q tile] softmax x passed the handover key of its exp2 pass of key tile j
   uint64_t o_full;    // MMA -> epilogue: the last PV completed
   uint64_t d_full;    // softmax (both warpgroups) -> epilogue: row sums published
   uint64_t drain[2];  // QK issuer, PV issuer: all own MMAs completed
   uint32_t tmem_base;
   int abort;
   float sv[kD];
-  float mrow[2][2][kTile];  // [Q tile][key tile % 2][row]: running max after that tile (log2 domain)
+  float arow[2][2][kTile];  // [Q tile][key tile % 2][row]: alpha of that tile
   float dsum[2][kTile];     // [Q tile][row]: sum of 448*p relative to the final max
 };
 static_assert(sizeof(AttnSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
@@ -110,8 +144,7 @@ static_assert(sizeof(AttnSmem) + 1024 <= 227 * 1024, "shared memory per CTA");
 // Wait-site identifiers recorded in the status detail word.
 enum : int {
   kSiteProdKEmpty = 1, kSiteProdVEmpty, kSiteMmaQ, kSiteMmaK, kSiteMmaP, kSiteMmaO, kSiteMmaV, kSiteMmaS,
-  kSiteSoftS, kSiteSoftM /* unused: the running max no longer crosses warpgroups; kept so ids stay fixed */,
-  kSiteSoftPV, kSiteCorrM, kSiteCorrPV, kSiteEpi, kSiteSoftTok
+  kSiteSoftS, kSiteSoftTok, kSiteSoftPV, kSiteCorrA, kSiteCorrPV, kSiteEpi
 };
 
 __device__ void record_failure(DevStatus* st, int code, int site, volatile int* abort) {
@@ -134,27 +167,28 @@ constexpr float kLog2_448 = 8.80735492205760410749f;
 #define H3ATTN_FMA_EXP2_PAIRS_OF_8 0
 #endif
 constexpr int kFmaExp2PairsOf8 = H3ATTN_FMA_EXP2_PAIRS_OF_8;
+static_assert(!(kFoldArg && kFmaExp2PairsOf8 != 0), "the FMA-pipe exp2 pairs need pre_turn");
 
-// Row maxima of the two 64-key halves (one K scale each) of the 128 FP32
-// scores of a row (integer-valued: the exact INT32 dot products), with 3-input
-// max; with kMasked, columns >= valid (keys past Tkv) are ignored.
-template <bool kMasked>
-__device__ __forceinline__ void rowmax128(const uint32_t (&s)[128], int valid, float& xm0, float& xm1) {
-  float m[8];
+// Maximum of the 64 FP32 scores s[OFF, OFF + 64) of one 64-key half (integer-valued:
+// the exact INT32 dot products); with kMasked, keys e >= valid (counted from the
+// half's first key; keys past Tkv) are ignored.  The maximum is exact in any order; it
+// is taken as a balanced tree of 3-input maxima (64 -> 22 -> 8 -> 4 -> 2 -> 1), the
+// mask applied where each score is used so that no masked copy is kept.
+template <bool kMasked, int OFF>
+__device__ __forceinline__ float rowmax64(const uint32_t (&s)[128], int valid) {
+  const auto v = [&](int e) {
+    const float a = __uint_as_float(s[OFF + e]);
+    return kMasked && e >= valid ? -INFINITY : a;
+  };
+  float l1[22], l2[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) m[c] = -INFINITY;
+  for (int k = 0; k < 21; ++k) l1[k] = fmax3(v(3 * k), v(3 * k + 1), v(3 * k + 2));
+  l1[21] = v(63);
 #pragma unroll
-  for (int e = 0; e < 128; e += 2) {
-    const int c = ((e >> 1) & 3) + (e >= 64 ? 4 : 0);
-    float a = __uint_as_float(s[e]), b = __uint_as_float(s[e + 1]);
-    if (kMasked) {
-      if (e >= valid) a = -INFINITY;
-      if (e + 1 >= valid) b = -INFINITY;
-    }
-    m[c] = fmax3(m[c], a, b);
-  }
-  xm0 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-  xm1 = fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7]));
+  for (int k = 0; k < 7; ++k) l2[k] = fmax3(l1[3 * k], l1[3 * k + 1], l1[3 * k + 2]);
+  l2[7] = l1[21];
+  const float a = fmax3(l2[0], l2[1], l2[2]), b = fmax3(l2[3], l2[4], l2[5]);
+  return fmaxf(fmax3(a, b, l2[6]), l2[7]);
 }
 
 // 2^u for a pair of arguments on the FMA pipe instead of the MUFU unit
@@ -183,7 +217,6 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
   q1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
 }
 
-
 // Softmax arithmetic of one row (128 keys, one per register), in two parts so that
 // only MUFU work needs the MUFU turn:
 //   pre_turn   in place, before the turn: u = s*f - mq (FP32 FMA; mq = m - log2(448),
@@ -193,7 +226,8 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
 //              into acc2 and the E4M3 words of q into w (4 keys per word); with
 //              kMasked, keys >= valid give 0.  The sums and conversions of every pair
 //              fill the MUFU latency.  The MUFU exp2 is volatile so that it stays
-//              after the turn's wait.
+//              after the turn's wait.  At key kTurnHandoverKey it arrives on tok, the
+//              other warpgroup's turn.
 __device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1, float mq) {
   const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
   const uint64_t negm = f2_pack(-mq, -mq);
@@ -214,15 +248,21 @@ __device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1,
 }
 
 template <bool kMasked>
-__device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, uint64_t (&acc2)[4],
-                                         uint32_t (&w)[32]) {
+__device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
+                                         uint64_t (&acc2)[4], uint32_t (&w)[32], uint64_t* tok) {
+  const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
+  const uint64_t negm = f2_pack(-mq, -mq);
 #pragma unroll
   for (int e = 0; e < 128; e += 4) {
+    if (e == kTurnHandoverKey) mbar_arrive(tok);
     uint32_t half[2];
+    float qq[4];
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int i = e + 2 * hp;
       float q0 = __uint_as_float(x[i]), q1 = __uint_as_float(x[i + 1]);
+      if (kFoldArg)  // u = s*f - mq here instead of in pre_turn (same FMA, same rounding)
+        f2_unpack(f2_fma(f2_pack(q0, q1), i < 64 ? ff0 : ff1, negm), q0, q1);
       if (((i >> 1) & 7) >= kFmaExp2PairsOf8) {
         asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
         asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
@@ -232,10 +272,16 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, ui
         if (i + 1 >= valid) q1 = 0.0f;
       }
       acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(q0, q1));
-      half[hp] = cvt_e4m3x2(q0, q1);
+      if (kCvtX4) {
+        qq[2 * hp] = q0;
+        qq[2 * hp + 1] = q1;
+      } else {
+        half[hp] = cvt_e4m3x2(q0, q1);
+      }
     }
-    w[e >> 2] = half[0] | (half[1] << 16);
+    w[e >> 2] = kCvtX4 ? cvt_e4m3x4_half_up(qq[0], qq[1], qq[2], qq[3]) : half[0] | (half[1] << 16);
   }
+  if (kTurnHandoverKey == 128) mbar_arrive(tok);
 }
 
 // End of every role: all 512 threads meet, then warp 1 frees the tensor memory.
@@ -252,21 +298,21 @@ __device__ __forceinline__ void attn_teardown(uint32_t tmem, bool owner) {
 // trace[(event * 2 + slot) * nkv + j]; slot = Q tile (0 = A, 1 = B) of the pair.
 enum : int {
   kEvSReady = 0,   // softmax warp: scores of key tile j ready (after the wait)
-  kEvMPub = 1,     // softmax warp: running max of tile j published to the correction
+  kEvAPub = 1,     // softmax warp: alpha of tile j published to the correction
   kEvPDone = 2,    // softmax warp: probabilities stored, MMA issuer signalled
   kEvQK = 3,       // MMA issuer: QK of key tile j issued
   kEvPV = 4,       // MMA issuer: PV of key tile j issued
   kEvCorr = 5,     // correction warp: O rescaled (or left alone), MMA issuer signalled
   kEvKFull = 6,    // MMA issuer: K tile j landed in shared memory (slot 0)
-  kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed
+  kEvProbs = 7,    // softmax warp: probabilities and their E4M3 words computed (end of the pass)
   kEvPVDone = 8,   // MMA issuer: PV of key tile j issued and committed
-  kEvSFree = 9,    // MMA issuer: scores of key tile j released (QK of tile j+1 may start)
-  kEvLd = 10,      // softmax warp: scores in registers
-  kEvMax = 11,     // softmax warp: own row maxima known
+  kEvSFree = 9,    // MMA issuer: scores of key tile j-1 released (QK of tile j may start)
+  kEvLd = 10,      // softmax warp: scores in registers (score buffer released)
+  kEvMax = 11,     // softmax warp: row maximum known
   kEvPFree = 12,   // softmax warp: probability buffer free (PV of tile j-1 completed)
   kEvPVP = 13,     // MMA issuer: probabilities of key tile j observed (p_full)
   kEvPVO = 14,     // MMA issuer: O ready for key tile j observed (o_ready)
-  kEvPDoneLast = 15,  // softmax warp of the last row quarter: probabilities handed over
+  kEvTurn = 15,    // softmax warp: MUFU turn taken (start of the pass)
   kNumEvents = 16
 };
 static_assert(kNumEvents == kTraceEvents, "trace buffer layout");
@@ -330,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[x], kTile);
       mbar_init(&sm.pv_done[x], 1);
       mbar_init(&sm.o_ready[x], kTile);
-      mbar_init(&sm.m_full[x][0], kTile);
-      mbar_init(&sm.m_full[x][1], kTile);
+      mbar_init(&sm.a_full[x][0], kTile);
+      mbar_init(&sm.a_full[x][1], kTile);
       mbar_init(&sm.tok[x], kTile);
     }
     mbar_init(&sm.o_full, 1);
@@ -437,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
               }
-              trace(kEvSFree, x, j - 1);
+              trace(kEvSFree, x, j);
             }
             tc_fence_after();
             // 8 MMAs of K = 16: BF16 key dims [16kk, 16kk+16) = bytes 32*(kk%4) of half kk/4
@@ -510,18 +556,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------- correction + epilogue ----
     regs_dealloc<kRegsCorrection>();
     bool ok = true;
-    float m_prev[2] = {-INFINITY, -INFINITY};  // running max of each Q tile after key tile j-1
     for (int j = 0; ok && j < nkv; ++j) {
       for (int x = 0; x < 2; ++x) {
-        ok = mbar_wait(&sm.m_full[x][j & 1], (uint32_t)(j >> 1) & 1u, abort, p.wait_limit_ns);
+        ok = mbar_wait(&sm.a_full[x][j & 1], (uint32_t)(j >> 1) & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
-          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrM, abort);
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteCorrA, abort);
           break;
         }
-        const float m_j = sm.mrow[x][j & 1][row];
-        const float alpha = ex2_approx(__fsub_rn(m_prev[x], m_j));
-        m_prev[x] = m_j;
+        const float alpha = sm.arow[x][j & 1][row];
         if (j > 0) {
           // O(x) holds the sum over key tiles < j once PV(x, j-1) has completed;
           // the wait also retires the previous phase of o_ready[x].
@@ -608,8 +651,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t prow = smem_u32(sm.p[x]) + (uint32_t)row * 128u;
     float m_w = -INFINITY, d_w = 0.0f;  // running max after the previous key tile, its row sum
     float sk0 = __ldg(skh), sk1 = __ldg(skh + 1);
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    // One key tile; false when a wait gave up (the failure is recorded).  Only the
+    // last tile can have keys past Tkv: it runs the masked instantiation after the
+    // loop, so the loop body holds one copy of the unrolled code.
+    const auto tile = [&](const int j, auto masked) -> bool {
+      constexpr bool kMasked = decltype(masked)::value;
+      bool ok;
       const float f0 = __fmul_rn(__fmul_rn(sqi, sk0), p.c_log2);
       const float f1 = __fmul_rn(__fmul_rn(sqi, sk1), p.c_log2);
       if (j + 1 < nkv) {
@@ -620,63 +667,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
         if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
-        break;
+        return false;
       }
       tc_fence_after();
       const bool tr = kTrace && tracing && quarter == 0 && lane == 0;
       if (tr) trace(kEvSReady, x, j);
-      const int valid = min(kTile, p.Tkv - j * kTile);
+      const int valid = kMasked ? p.Tkv - j * kTile : kTile;
+      // scores: keys [0,64) loaded and waited for, keys [64,128) in flight while the
+      // first half's maximum is taken
       uint32_t xs[128];
-      tmem_ld64x2(tS, xs);
+      tmem_ld64_wait_at<0>(tS, xs);
+      tmem_ld64_async_at<64>(tS + 64u, xs);
+      const float xm0 = kMasked && valid < 64 ? rowmax64<true, 0>(xs, valid) : rowmax64<false, 0>(xs, valid);
+      tmem_wait_ld_at<64>(xs);
       tc_fence_before();
-      mbar_arrive(&sm.s_free[x]);
+      mbar_arrive(&sm.s_free[x]);  // QK of the next key tile may overwrite S(x)
       if (tr) trace(kEvLd, x, j);
-      float xm0, xm1;
-      if (valid < kTile)
-        rowmax128<true>(xs, valid, xm0, xm1);
-      else
-        rowmax128<false>(xs, valid, xm0, xm1);
-      const float t0m = __fmul_rn(xm0, f0);  // valid >= 1: half 0 has a key
+      const float xm1 =
+          kMasked ? rowmax64<true, 64>(xs, valid - 64) : rowmax64<false, 64>(xs, valid - 64);
+      const float t0m = __fmul_rn(xm0, f0);                           // valid >= 1: half 0 has a key
       const float t1m = valid > 64 ? __fmul_rn(xm1, f1) : -INFINITY;
+      const float m_j = fmaxf(m_w, fmaxf(t0m, t1m));
       if (tr) {
-        asm volatile("" ::"f"(t0m), "f"(t1m));  // the maxima exist before the stamp is taken
+        asm volatile("" ::"f"(m_j));  // the maximum exists before the stamp is taken
         trace(kEvMax, x, j);
       }
-      const float m_j = fmaxf(m_w, fmaxf(t0m, t1m));
-      sm.mrow[x][j & 1][row] = m_j;
-      mbar_arrive(&sm.m_full[x][j & 1]);
-      if (tr) trace(kEvMPub, x, j);
       uint32_t pw[32];
       uint64_t acc2[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
       const float mq = __fsub_rn(m_j, kLog2_448);
-      pre_turn(xs, f0, f1, mq);
-      // MUFU turn: the exp2 passes alternate A(0) B(0) A(1) B(1) ... so that
-      // each runs with the MUFU unit to itself while the other warpgroup does
-      // the rest of its tile.
+      if (!kFoldArg) pre_turn(xs, f0, f1, mq);
+      // MUFU turn: the exp2 passes start in turn A(0) B(0) A(1) B(1) ..., each
+      // after the other warpgroup's pass has reached its handover key, so that
+      // a pass has the MUFU unit (nearly) to itself while the other warpgroup
+      // does the rest of its tile.
       if (x == 1 || j >= 1) {
         const int jt = x == 1 ? j : j - 1;  // A waits for B's pass of j-1, B for A's pass of j
         ok = mbar_wait(&sm.tok[1 - x], (uint32_t)jt & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftTok, abort);
-          break;
+          return false;
         }
       }
-      if (valid < kTile)
-        probs128<true>(xs, valid, acc2, pw);
-      else
-        probs128<false>(xs, valid, acc2, pw);
-      mbar_arrive(&sm.tok[x]);
+      if (tr) trace(kEvTurn, x, j);
+      // the rescale factor of this tile, on MUFU inside the turn (2^-inf = 0 on the first tile)
+      float alpha;
+      asm volatile("ex2.approx.f32 %0, %1;" : "=f"(alpha) : "f"(__fsub_rn(m_w, m_j)));
+      probs128<kMasked>(xs, valid, f0, f1, mq, acc2, pw, &sm.tok[x]);
       if (tr) trace(kEvProbs, x, j);
+      sm.arow[x][j & 1][row] = alpha;
+      mbar_arrive(&sm.a_full[x][j & 1]);
+      if (tr) trace(kEvAPub, x, j);
       if (j >= 1) {
         // the probability buffer still feeds PV(x, j-1) until that MMA has completed
         ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
           if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftPV, abort);
-          break;
+          return false;
         }
         if (tr) trace(kEvPFree, x, j);
       }
@@ -688,14 +738,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&sm.p_full[x]);
       if (tr) trace(kEvPDone, x, j);
-      if (kTrace && tracing && quarter == 3 && lane == 0) trace(kEvPDoneLast, x, j);
       float a[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
       const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-      d_w = __fadd_rn(__fmul_rn(d_w, ex2_approx(__fsub_rn(m_w, m_j))), es);
+      d_w = __fadd_rn(__fmul_rn(d_w, alpha), es);
       m_w = m_j;
-    }
+      return true;
+    };
+    const int full_tiles = p.Tkv % kTile == 0 ? nkv : nkv - 1;  // tiles whose 128 keys are all valid
+    bool ok = true;
+    for (int j = 0; ok && j < full_tiles; ++j) ok = tile(j, std::false_type{});
+    if (ok && full_tiles < nkv) ok = tile(nkv - 1, std::true_type{});
     if (ok) {
       sm.dsum[x][row] = d_w;
       mbar_arrive(&sm.d_full);

@@ -27,7 +27,7 @@ SITE_PV_O_READY = 6                      # PV issuer waiting for "O ready"
 SITE_QK_S_FREE = 8                       # QK issuer waiting for a free score buffer
 SITE_SOFTMAX_PV = 11                     # softmax waiting for its probability buffer
 SITE_CORR_PV = 13                        # correction waiting for PV of the previous tile
-SITE_SOFTMAX_TURN = 15                   # softmax waiting for its MUFU turn
+SITE_SOFTMAX_TURN = 10                   # softmax waiting for its MUFU turn
 SMALL_SITES = {SITE_PV_O_READY, SITE_SOFTMAX_PV, SITE_CORR_PV}
 LARGE_SITES = SMALL_SITES | {SITE_K_PRODUCER, SITE_V_PRODUCER, SITE_QK_S_FREE, SITE_SOFTMAX_TURN}
 LIMIT_NS = 20_000_000  # 20 ms
