@@ -74,6 +74,11 @@ __device__ __forceinline__ uint32_t col_o(int x) { return 256u + 128u * (uint32_
 #define H3ATTN_TURN_HANDOVER_KEY 64
 #endif
 constexpr int kTurnHandoverKey = H3ATTN_TURN_HANDOVER_KEY;
+// Key of the exp2 pass at which the barriers the rest of the tile (and the next one)
+// depends on are tested without blocking: a blocking test of an already-completed
+// phase still costs the barrier round trip on the chain between two passes, which
+// these tests instead overlap with the pass.
+constexpr int kMidPassKey = 96;
 // 1: the exp2 arguments u = s*f - mq are formed inside the exp2 pass, next to each
 // exp2; 0: in place before the pass (pre_turn).  Either gives the same bits.
 #ifndef H3ATTN_FOLD_ARG
@@ -167,7 +172,13 @@ constexpr float kLog2_448 = 8.80735492205760410749f;
 #define H3ATTN_FMA_EXP2_PAIRS_OF_8 0
 #endif
 constexpr int kFmaExp2PairsOf8 = H3ATTN_FMA_EXP2_PAIRS_OF_8;
-static_assert(!(kFoldArg && kFmaExp2PairsOf8 != 0), "the FMA-pipe exp2 pairs need pre_turn");
+// Packed FP32-pair partial sums of each row's probabilities (4: partial k holds the pairs
+// (2i, 2i+1) with i = k mod 4; 8: i = k mod 8).
+#ifndef H3ATTN_SUM_ACC
+#define H3ATTN_SUM_ACC 4
+#endif
+constexpr int kSumAcc = H3ATTN_SUM_ACC;
+static_assert(kSumAcc == 4 || kSumAcc == 8, "row-sum partials");
 
 // Maximum of the 64 FP32 scores s[OFF, OFF + 64) of one 64-key half (integer-valued:
 // the exact INT32 dot products); with kMasked, keys e >= valid (counted from the
@@ -227,7 +238,8 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
 //              kMasked, keys >= valid give 0.  The sums and conversions of every pair
 //              fill the MUFU latency.  The MUFU exp2 is volatile so that it stays
 //              after the turn's wait.  At key kTurnHandoverKey it arrives on tok, the
-//              other warpgroup's turn.
+//              other warpgroup's turn; at key kMidPassKey it runs mid_pass (the
+//              early barrier tests of the tile).
 __device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1, float mq) {
   const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
   const uint64_t negm = f2_pack(-mq, -mq);
@@ -247,23 +259,31 @@ __device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1,
   for (int i = 0; i < 128; ++i) asm volatile("" : "+r"(x[i]));
 }
 
-template <bool kMasked>
+template <bool kMasked, typename MidPass>
 __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, float f0, float f1, float mq,
-                                         uint64_t (&acc2)[4], uint32_t (&w)[32], uint64_t* tok) {
+                                         uint64_t (&acc2)[kSumAcc], uint32_t (&w)[32], uint64_t* tok,
+                                         const MidPass& mid_pass) {
   const uint64_t ff0 = f2_pack(f0, f0), ff1 = f2_pack(f1, f1);
   const uint64_t negm = f2_pack(-mq, -mq);
 #pragma unroll
   for (int e = 0; e < 128; e += 4) {
     if (e == kTurnHandoverKey) mbar_arrive(tok);
+    if (e == kMidPassKey) mid_pass();
     uint32_t half[2];
     float qq[4];
 #pragma unroll
     for (int hp = 0; hp < 2; ++hp) {
       const int i = e + 2 * hp;
       float q0 = __uint_as_float(x[i]), q1 = __uint_as_float(x[i + 1]);
-      if (kFoldArg)  // u = s*f - mq here instead of in pre_turn (same FMA, same rounding)
-        f2_unpack(f2_fma(f2_pack(q0, q1), i < 64 ? ff0 : ff1, negm), q0, q1);
-      if (((i >> 1) & 7) >= kFmaExp2PairsOf8) {
+      const bool fma_pair = ((i >> 1) & 7) < kFmaExp2PairsOf8;
+      if (kFoldArg) {  // u = s*f - mq here instead of in pre_turn (same FMA, same rounding)
+        const uint64_t u = f2_fma(f2_pack(q0, q1), i < 64 ? ff0 : ff1, negm);
+        if (fma_pair)
+          exp2_fma_pair(u, q0, q1);
+        else
+          f2_unpack(u, q0, q1);
+      }
+      if (!fma_pair) {
         asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
         asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
       }
@@ -271,7 +291,7 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
         if (i >= valid) q0 = 0.0f;
         if (i + 1 >= valid) q1 = 0.0f;
       }
-      acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(q0, q1));
+      acc2[(i >> 1) & (kSumAcc - 1)] = f2_add(acc2[(i >> 1) & (kSumAcc - 1)], f2_pack(q0, q1));
       if (kCvtX4) {
         qq[2 * hp] = q0;
         qq[2 * hp + 1] = q1;
@@ -654,20 +674,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One key tile; false when a wait gave up (the failure is recorded).  Only the
     // last tile can have keys past Tkv: it runs the masked instantiation after the
     // loop, so the loop body holds one copy of the unrolled code.
+    // Outcomes of the early (non-blocking) barrier tests, carried to where each barrier
+    // is needed; a test that found its phase incomplete falls back to the blocking wait.
+    bool s_seen = false;    // scores of this tile's key tile already seen complete
+    bool tok_seen = false;  // this tile's MUFU turn already seen granted
     const auto tile = [&](const int j, auto masked) -> bool {
       constexpr bool kMasked = decltype(masked)::value;
-      bool ok;
+      bool ok = true;
       const float f0 = __fmul_rn(__fmul_rn(sqi, sk0), p.c_log2);
       const float f1 = __fmul_rn(__fmul_rn(sqi, sk1), p.c_log2);
-      if (j + 1 < nkv) {
-        sk0 = __ldg(skh + 2 * (j + 1));
-        sk1 = __ldg(skh + 2 * (j + 1) + 1);
+      if (j + 1 < nkv) {  // the next tile's K scales, a tile ahead of their use
+        sk0 = ldg_f32_issued_here(skh + 2 * (j + 1));
+        sk1 = ldg_f32_issued_here(skh + 2 * (j + 1) + 1);
       }
-      ok = mbar_wait(&sm.s_full[x], (uint32_t)j & 1u, abort, p.wait_limit_ns);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) {
-        if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
-        return false;
+      if (!s_seen) {
+        ok = mbar_wait(&sm.s_full[x], (uint32_t)j & 1u, abort, p.wait_limit_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0) record_failure(p.status, H3ATTN_ERR_TIMEOUT, kSiteSoftS, abort);
+          return false;
+        }
       }
       tc_fence_after();
       const bool tr = kTrace && tracing && quarter == 0 && lane == 0;
@@ -693,16 +719,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         trace(kEvMax, x, j);
       }
       uint32_t pw[32];
-      uint64_t acc2[4];
+      uint64_t acc2[kSumAcc];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc2[i] = 0ull;
+      for (int i = 0; i < kSumAcc; ++i) acc2[i] = 0ull;
       const float mq = __fsub_rn(m_j, kLog2_448);
       if (!kFoldArg) pre_turn(xs, f0, f1, mq);
       // MUFU turn: the exp2 passes start in turn A(0) B(0) A(1) B(1) ..., each
       // after the other warpgroup's pass has reached its handover key, so that
       // a pass has the MUFU unit (nearly) to itself while the other warpgroup
       // does the rest of its tile.
-      if (x == 1 || j >= 1) {
+      if ((x == 1 || j >= 1) && !tok_seen) {
         const int jt = x == 1 ? j : j - 1;  // A waits for B's pass of j-1, B for A's pass of j
         ok = mbar_wait(&sm.tok[1 - x], (uint32_t)jt & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -715,12 +741,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the rescale factor of this tile, on MUFU inside the turn (2^-inf = 0 on the first tile)
       float alpha;
       asm volatile("ex2.approx.f32 %0, %1;" : "=f"(alpha) : "f"(__fsub_rn(m_w, m_j)));
-      probs128<kMasked>(xs, valid, f0, f1, mq, acc2, pw, &sm.tok[x]);
+      // mid-pass: test the probability buffer (PV of tile j-1) and the next tile's scores
+      bool p_seen = j == 0;
+      s_seen = false;
+      const auto mid_pass = [&]() {
+        if (j >= 1) p_seen = mbar_test(&sm.pv_done[x], (uint32_t)(j - 1) & 1u);
+        if (j + 1 < nkv) s_seen = mbar_test(&sm.s_full[x], (uint32_t)(j + 1) & 1u);
+      };
+      probs128<kMasked>(xs, valid, f0, f1, mq, acc2, pw, &sm.tok[x], mid_pass);
       if (tr) trace(kEvProbs, x, j);
       sm.arow[x][j & 1][row] = alpha;
       mbar_arrive(&sm.a_full[x][j & 1]);
       if (tr) trace(kEvAPub, x, j);
-      if (j >= 1) {
+      if (!p_seen) {
         // the probability buffer still feeds PV(x, j-1) until that MMA has completed
         ok = mbar_wait(&sm.pv_done[x], (uint32_t)(j - 1) & 1u, abort, p.wait_limit_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -738,9 +771,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&sm.p_full[x]);
       if (tr) trace(kEvPDone, x, j);
-      float a[8];
+      // the next tile's MUFU turn, tested now so that its round trip overlaps the row sum
+      tok_seen = false;
+      if (j + 1 < nkv) {
+        const int jt = x == 1 ? j + 1 : j;
+        tok_seen = mbar_test(&sm.tok[1 - x], (uint32_t)jt & 1u);
+      }
+      float a[2 * kSumAcc];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
+      for (int i = 0; i < kSumAcc; ++i) f2_unpack(acc2[i], a[2 * i], a[2 * i + 1]);
+      if (kSumAcc == 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = a[i] + a[i + 8];
+      }
       const float es = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
       d_w = __fadd_rn(__fmul_rn(d_w, alpha), es);
       m_w = m_j;

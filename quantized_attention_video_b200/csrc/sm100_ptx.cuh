@@ -55,6 +55,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (acquire at CTA scope on
+// success): its latency overlaps whatever the thread issues before it uses the result.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait that lets the hardware suspend the thread for up to hint_ns while
 // the phase is incomplete (it resumes when the phase completes), so waiting
 // warps do not spin on the issue slots the working warps need.
@@ -225,6 +239,15 @@ __device__ __forceinline__ void tmem_wait_ld_at(uint32_t (&r)[128]) {
                : "+r"(r[OFF + 0]), "+r"(r[OFF + 1]), "+r"(r[OFF + 2]), "+r"(r[OFF + 3]), "+r"(r[OFF + 4]), "+r"(r[OFF + 5]), "+r"(r[OFF + 6]), "+r"(r[OFF + 7]), "+r"(r[OFF + 8]), "+r"(r[OFF + 9]), "+r"(r[OFF + 10]), "+r"(r[OFF + 11]), "+r"(r[OFF + 12]), "+r"(r[OFF + 13]), "+r"(r[OFF + 14]), "+r"(r[OFF + 15]), "+r"(r[OFF + 16]), "+r"(r[OFF + 17]), "+r"(r[OFF + 18]), "+r"(r[OFF + 19]), "+r"(r[OFF + 20]), "+r"(r[OFF + 21]), "+r"(r[OFF + 22]), "+r"(r[OFF + 23]), "+r"(r[OFF + 24]), "+r"(r[OFF + 25]), "+r"(r[OFF + 26]), "+r"(r[OFF + 27]), "+r"(r[OFF + 28]), "+r"(r[OFF + 29]), "+r"(r[OFF + 30]), "+r"(r[OFF + 31]), "+r"(r[OFF + 32]), "+r"(r[OFF + 33]), "+r"(r[OFF + 34]), "+r"(r[OFF + 35]), "+r"(r[OFF + 36]), "+r"(r[OFF + 37]), "+r"(r[OFF + 38]), "+r"(r[OFF + 39]), "+r"(r[OFF + 40]), "+r"(r[OFF + 41]), "+r"(r[OFF + 42]), "+r"(r[OFF + 43]), "+r"(r[OFF + 44]), "+r"(r[OFF + 45]), "+r"(r[OFF + 46]), "+r"(r[OFF + 47]), "+r"(r[OFF + 48]), "+r"(r[OFF + 49]), "+r"(r[OFF + 50]), "+r"(r[OFF + 51]), "+r"(r[OFF + 52]), "+r"(r[OFF + 53]), "+r"(r[OFF + 54]), "+r"(r[OFF + 55]), "+r"(r[OFF + 56]), "+r"(r[OFF + 57]), "+r"(r[OFF + 58]), "+r"(r[OFF + 59]), "+r"(r[OFF + 60]), "+r"(r[OFF + 61]), "+r"(r[OFF + 62]), "+r"(r[OFF + 63])
                :
                : "memory");
+}
+
+// A read-only FP32 global load issued where it stands in the program (a volatile asm
+// statement): the compiler may not sink it to its first use, so a load issued one loop
+// iteration ahead of that use keeps its latency off the iteration's critical path.
+__device__ __forceinline__ float ldg_f32_issued_here(const float* ptr) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(ptr) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------ packed FP32 pairs ----
