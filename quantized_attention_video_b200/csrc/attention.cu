@@ -236,8 +236,11 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t u, float& q0, float& q1) 
 //   probs128   in the turn: q = 2^u on MUFU for the other pairs, FP32 partial sums of q
 //              into acc2 and the E4M3 words of q into w (4 keys per word); with
 //              kMasked, keys >= valid give 0.  The sums and conversions of every pair
-//              fill the MUFU latency.  The MUFU exp2 is volatile so that it stays
-//              after the turn's wait.  At key kTurnHandoverKey it arrives on tok, the
+//              fill the MUFU latency.  Every exp2 stays after the turn's wait: with
+//              kFoldArg through its arguments (mq, f0 and f1 are redefined after the
+//              wait), which leaves the compiler free to interleave the exp2s with the
+//              other work of the pass; without it, as a volatile instruction.  At key
+//              kTurnHandoverKey it arrives on tok, the
 //              other warpgroup's turn; at key kMidPassKey it runs mid_pass (the
 //              early barrier tests of the tile).
 __device__ __forceinline__ void pre_turn(uint32_t (&x)[128], float f0, float f1, float mq) {
@@ -284,8 +287,13 @@ __device__ __forceinline__ void probs128(const uint32_t (&x)[128], int valid, fl
           f2_unpack(u, q0, q1);
       }
       if (!fma_pair) {
-        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
-        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
+        if (kFoldArg) {  // ordered after the turn through its arguments (mq, f0, f1)
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
+          asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
+        } else {         // arguments formed before the turn: the exp2 itself stays after it
+          asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q0) : "f"(q0));
+          asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(q1) : "f"(q1));
+        }
       }
       if (kMasked) {
         if (i >= valid) q0 = 0.0f;
@@ -738,6 +746,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (tr) trace(kEvTurn, x, j);
+      // The exp2 instructions are not volatile, so that the compiler can interleave them
+      // with the sums and conversions of earlier keys; their arguments come from copies
+      // of mq, f0 and f1 that this empty volatile statement redefines after the turn's
+      // wait, which keeps every exp2 of the pass after the wait.
+      float mq_t = mq, f0_t = f0, f1_t = f1;
+      asm volatile("" : "+f"(mq_t), "+f"(f0_t), "+f"(f1_t));
       // the rescale factor of this tile, on MUFU inside the turn (2^-inf = 0 on the first tile)
       float alpha;
       asm volatile("ex2.approx.f32 %0, %1;" : "=f"(alpha) : "f"(__fsub_rn(m_w, m_j)));
@@ -748,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1) p_seen = mbar_test(&sm.pv_done[x], (uint32_t)(j - 1) & 1u);
         if (j + 1 < nkv) s_seen = mbar_test(&sm.s_full[x], (uint32_t)(j + 1) & 1u);
       };
-      probs128<kMasked>(xs, valid, f0, f1, mq, acc2, pw, &sm.tok[x], mid_pass);
+      probs128<kMasked>(xs, valid, f0_t, f1_t, mq_t, acc2, pw, &sm.tok[x], mid_pass);
       if (tr) trace(kEvProbs, x, j);
       sm.arow[x][j & 1][row] = alpha;
       mbar_arrive(&sm.a_full[x][j & 1]);
