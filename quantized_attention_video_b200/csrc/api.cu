@@ -11,6 +11,51 @@
 
 using namespace h3;
 
+uint64_t h3::current_context_id() {
+  typedef int (*GetCurrentFn)(void**);
+  typedef int (*GetIdFn)(void*, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != 0 || ctx == nullptr || get_id(ctx, &id) != 0) return 0;
+  return (uint64_t)id;
+}
+
+namespace {
+std::mutex g_context_set_mu;
+}  // namespace
+
+bool h3::ContextSet::contains(uint64_t id) {
+  if (id == 0) return false;
+  std::lock_guard<std::mutex> lk(g_context_set_mu);
+  for (int i = 0; i < n_; ++i)
+    if (ids_[i] == id) return true;
+  return false;
+}
+
+void h3::ContextSet::add(uint64_t id) {
+  if (id == 0) return;
+  std::lock_guard<std::mutex> lk(g_context_set_mu);
+  for (int i = 0; i < n_; ++i)
+    if (ids_[i] == id) return;
+  ids_[next_] = id;  // beyond 64 contexts the oldest record is dropped (its attributes are then set again)
+  next_ = (next_ + 1) % 64;
+  if (n_ < 64) ++n_;
+}
+
 namespace {
 
 constexpr double kLog2e = 1.44269504088896340736;

@@ -928,14 +928,9 @@ constexpr size_t kAttnSmemBytes = sizeof(AttnSmem) + 1024;
 constexpr size_t kDebugSmemBytes = sizeof(DebugSmem) + 1024;
 
 cudaError_t ensure_attrs() {
-  static int done_mask = 0;  // one bit per device ordinal < 32
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lk(mu);
-  if (dev < 32 && (done_mask >> dev) & 1) return cudaSuccess;
-  e = cudaFuncSetAttribute(attn_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
+  static ContextSet done;  // contexts whose attributes are set
+  if (done.contains(current_context_id())) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(attn_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmemBytes);
   if (e != cudaSuccess) return e;
@@ -948,7 +943,7 @@ cudaError_t ensure_attrs() {
     if (e != cudaSuccess) return e;
     if ((int64_t)fa.numRegs * kThreads < kRegSplitTotal) return cudaErrorInvalidConfiguration;
   }
-  if (dev < 32) done_mask |= 1 << dev;
+  done.add(current_context_id());  // the calls above made the device's primary context current if none was
   return cudaSuccess;
 }
 

@@ -100,6 +100,26 @@ cudaError_t launch_attention(const char* ws, const Shape& s, const Layout& L, fl
                              uint64_t* trace = nullptr, int trace_block = -1,
                              uint64_t wait_limit_ns = kDefaultWaitLimitNs, bool withhold_o_ready = false);
 constexpr int kTraceEvents = 16;  // events per (tile slot, key tile) in the timeline trace
+
+// Kernel attributes (cudaFuncSetAttribute) belong to a CUDA context, so a record of the
+// contexts whose attributes are set must name contexts, not device ordinals: after a
+// cudaDeviceReset, or with another context made current on the same device, the
+// attributes have to be set again.  current_context_id() is the driver's id of the
+// context current on this thread (unique for the life of the process; cuCtxGetId), or
+// 0 when there is none or the driver cannot tell, in which case nothing is recorded.
+uint64_t current_context_id();
+
+// A thread-safe record of the contexts that have been set up.
+class ContextSet {
+ public:
+  bool contains(uint64_t id);
+  void add(uint64_t id);  // ignores id 0
+
+ private:
+  uint64_t ids_[64] = {};
+  int n_ = 0;
+  int next_ = 0;
+};
 cudaError_t launch_debug_qk(const char* ws, const Shape& s, const Layout& L, int b, int h, int qt, int kt,
                             int32_t* out, cudaStream_t st, h3attn_status* why);
 

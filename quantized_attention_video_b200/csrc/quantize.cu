@@ -661,18 +661,13 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(const uint16_t* x, int64
   }
 }
 
-// The finalize kernel's shared memory is above the default 48 KB limit (set once per device).
+// The finalize kernel's shared memory is above the default 48 KB limit (set once per context).
 cudaError_t ensure_prep_attrs() {
-  static int done_mask = 0;  // one bit per device ordinal < 32
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static ContextSet done;  // contexts whose attribute is set
+  if (done.contains(current_context_id())) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinSmemBytes);
   if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lk(mu);
-  if (dev < 32 && (done_mask >> dev) & 1) return cudaSuccess;
-  e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinSmemBytes);
-  if (e != cudaSuccess) return e;
-  if (dev < 32) done_mask |= 1 << dev;
+  done.add(current_context_id());
   return cudaSuccess;
 }
 

@@ -9,6 +9,7 @@
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <cuda_runtime.h>
 
@@ -16,22 +17,11 @@
 
 static int read_all(FILE* f, void* p, size_t n) { return fread(p, 1, n, f) == n; }
 
-int main(int argc, char** argv) {
-  if (argc != 3) {
-    fprintf(stderr, "usage: %s input.bin output.bin\n", argv[0]);
-    return 1;
-  }
-  FILE* in = fopen(argv[1], "rb");
-  if (!in) return 1;
-  int32_t dims[4];
-  float scale;
-  if (!read_all(in, dims, sizeof dims) || !read_all(in, &scale, sizeof scale)) return 1;
-  const int B = dims[0], Tq = dims[1], Tkv = dims[2], H = dims[3], D = H3ATTN_HEAD_DIM;
+/* One forward pass of the problem in host[] (Q, K, V dense) into out_host[]: allocates the
+ * device buffers, uploads, runs, checks the device status, downloads and frees. */
+static int run_once(const uint16_t* host, int B, int Tq, int Tkv, int H, float scale, uint16_t* out_host) {
+  const int D = H3ATTN_HEAD_DIM;
   const size_t nq = (size_t)B * Tq * H * D, nkv = (size_t)B * Tkv * H * D;
-  uint16_t* host = (uint16_t*)malloc(2 * (nq + 2 * nkv));
-  if (!host || !read_all(in, host, 2 * (nq + 2 * nkv))) return 1;
-  fclose(in);
-
   const size_t ws_bytes = h3attn_workspace_bytes(B, Tq, Tkv, H, D);
   if (ws_bytes == 0) return 2 + H3ATTN_ERR_INVALID_ARG;
   void *dq, *dk, *dv, *dout, *ws;
@@ -59,16 +49,56 @@ int main(int argc, char** argv) {
     fprintf(stderr, "device status: %s\n", h3attn_status_string(st));
     return 2 + st;
   }
-  if (cudaMemcpy(host, dout, 2 * nq, cudaMemcpyDeviceToHost) != cudaSuccess) return 1;
-  FILE* o = fopen(argv[2], "wb");
-  if (!o || fwrite(host, 2, nq, o) != nq) return 1;
-  fclose(o);
+  if (cudaMemcpy(out_host, dout, 2 * nq, cudaMemcpyDeviceToHost) != cudaSuccess) return 1;
   cudaFree(dq);
   cudaFree(dk);
   cudaFree(dv);
   cudaFree(dout);
   cudaFree(ws);
+  return 0;
+}
+
+/* With a third argument "reset": after the first pass the program resets the device (which
+ * destroys its context and every allocation in it) and runs the pass again in the new
+ * context; the two outputs must be equal.  The library sets its kernels' shared-memory
+ * attributes once per context, so this checks that it notices the new context. */
+int main(int argc, char** argv) {
+  if (argc != 3 && !(argc == 4 && strcmp(argv[3], "reset") == 0)) {
+    fprintf(stderr, "usage: %s input.bin output.bin [reset]\n", argv[0]);
+    return 1;
+  }
+  FILE* in = fopen(argv[1], "rb");
+  if (!in) return 1;
+  int32_t dims[4];
+  float scale;
+  if (!read_all(in, dims, sizeof dims) || !read_all(in, &scale, sizeof scale)) return 1;
+  const int B = dims[0], Tq = dims[1], Tkv = dims[2], H = dims[3], D = H3ATTN_HEAD_DIM;
+  const size_t nq = (size_t)B * Tq * H * D, nkv = (size_t)B * Tkv * H * D;
+  uint16_t* host = (uint16_t*)malloc(2 * (nq + 2 * nkv));
+  uint16_t* result = (uint16_t*)malloc(2 * nq);
+  if (!host || !result || !read_all(in, host, 2 * (nq + 2 * nkv))) return 1;
+  fclose(in);
+
+  int rc = run_once(host, B, Tq, Tkv, H, scale, result);
+  if (rc != 0) return rc;
+  if (argc == 4) {
+    uint16_t* again = (uint16_t*)malloc(2 * nq);
+    if (!again) return 1;
+    if (cudaDeviceReset() != cudaSuccess) return 1;
+    rc = run_once(host, B, Tq, Tkv, H, scale, again);
+    if (rc != 0) return rc;
+    if (memcmp(again, result, 2 * nq) != 0) {
+      fprintf(stderr, "the output after the device reset differs\n");
+      return 1;
+    }
+    free(again);
+  }
+  FILE* o = fopen(argv[2], "wb");
+  if (!o || fwrite(result, 2, nq, o) != nq) return 1;
+  fclose(o);
   free(host);
-  printf("ok: B=%d Tq=%d Tkv=%d H=%d, library version %d\n", B, Tq, Tkv, H, h3attn_version());
+  free(result);
+  printf("ok: B=%d Tq=%d Tkv=%d H=%d, library version %d%s\n", B, Tq, Tkv, H, h3attn_version(),
+         argc == 4 ? ", again after a device reset" : "");
   return 0;
 }

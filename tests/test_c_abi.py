@@ -76,3 +76,29 @@ def test_c_program_matches_the_python_binding(tmp_path):
     assert h3.h3attn_check_status(ws) == h3.OK
     ref = out.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(got, ref)
+
+
+@pytest.mark.gpu
+def test_c_program_runs_again_after_a_device_reset(tmp_path):
+    """The program runs the forward pass, resets the device (a new context: every
+    allocation and every kernel attribute of the old one is gone) and runs it again: the
+    library must set its kernels' shared-memory attributes for the new context, and the
+    second output must equal the first (the program compares them) and the usual bytes."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    exe = build_program()
+    w = synth.WORKLOADS["fixed_q128_kv192"]
+    x = synth.make_inputs(w)
+    inp = tmp_path / "in.bin"
+    with open(inp, "wb") as f:
+        f.write(struct.pack("<4if", w.B, w.Tq, w.Tkv, w.H, w.scale))
+        for n in ("q", "k", "v"):
+            f.write(np.ascontiguousarray(x[n]).tobytes())
+    plain, again = tmp_path / "plain.bin", tmp_path / "again.bin"
+    r = subprocess.run([exe, str(inp), str(plain)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    r = subprocess.run([exe, str(inp), str(again), "reset"], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "after a device reset" in r.stdout
+    assert np.array_equal(np.fromfile(again, dtype=np.uint16), np.fromfile(plain, dtype=np.uint16))
