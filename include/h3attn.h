@@ -179,9 +179,9 @@ size_t h3attn_forward_host_bytes(int B, int Tq, int Tkv, int H, int D, int heads
  *     owned by the caller; holds the staging and the per-slot workspaces.
  * Asynchronous on `stream`; creates its two copy streams and eight events per call and
  * releases them before returning (the runtime frees them once their work is done).
- * Device-side status: h3attn_forward_host_check_status.  The zero-copy layout of the
- * north-star ("H3 Performance Roadmap", Phase 4 item 5: token-major in and out) applies
- * to the host views the same way. */
+ * Device-side status: h3attn_forward_host_check_status.  The zero-copy layout of
+ * "H3 Performance Roadmap", Phase 4 item 5 (token-major in and out) applies to the host
+ * views the same way. */
 h3attn_status h3attn_forward_host(const h3attn_bf16_view* q, const h3attn_bf16_view* k,
                                   const h3attn_bf16_view* v, int B, int Tq, int Tkv, int H, int D,
                                   float softmax_scale, const h3attn_bf16_out* out, int heads_per_group,
