@@ -65,10 +65,16 @@ def parse():
                     help="per-call latency of the fixed 128 x 192 shape by the pages' method (samples of 20 "
                          "back-to-back calls, p50 and CV), forward and attend-only samples alternated")
     ap.add_argument("--samples", type=int, default=500)
+    ap.add_argument("--ulysses", action="store_true",
+                    help="one sequence of the workload spread over the GPUs by tokens: head-sharding all-to-alls "
+                         "around the attention of H/N heads per GPU (strong scaling)")
     return ap.parse_args()
 
 
 def dist_env():
+    # NCCL prints its version banner on stdout unless told otherwise; the bench's stdout is
+    # its one JSON line
+    os.environ.setdefault("NCCL_DEBUG", "WARN")
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
 
 
@@ -454,6 +460,109 @@ def run_ours(args, w):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------- Ulysses mode ----
+def run_ulysses(args, w):
+    """One sequence of the workload spread over the ranks by tokens (strong scaling: the
+    whole job is one problem).  Each step: the token-to-head all-to-all of Q, K and V, the
+    library forward pass on this rank's H/N heads, the head-to-token all-to-all of the
+    output.  Inputs resident on the GPUs; CUDA events around each part, max over ranks."""
+    import dataclasses
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    import quantized_attention_video_b200 as h3
+    from quantized_attention_video_b200 import build as h3build
+    from quantized_attention_video_b200 import ulysses
+
+    if w.packed or w.norm_rope or w.Tq != w.Tkv:
+        raise SystemExit("--ulysses takes a self-attention workload in the separate layout")
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1 and "MASTER_ADDR" not in os.environ:
+        with socket.socket() as sck:
+            sck.bind(("127.0.0.1", 0))
+            port = sck.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if w.H % world:
+        raise SystemExit(f"{w.H} heads do not split over {world} GPUs")
+    if rank == 0 or not os.path.exists(h3build.SO):
+        h3build.build()
+    dist.barrier()
+    h3.lib()
+
+    x = synth.make_inputs(w)
+    counts = ulysses.token_counts(w.Tq, world)
+    off = sum(counts[:rank])
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x[n][:, off:off + counts[rank]]).view(np.int16)).to(dev)
+               .view(torch.bfloat16) for n in ("q", "k", "v"))
+    del x
+    hn = w.H // world
+    ws = h3.new_workspace(w.B, w.Tq, w.Tq, hn, device=dev)
+    oh = torch.empty(w.B, w.Tq, hn, w.D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        qh, kh, vh = ulysses.seq_to_head([q, k, v], w.Tq)
+        if ev:
+            ev[1].record(stream)
+        h3.h3attn_forward_ex(qh, kh, vh, w.scale, oh, ws, stream)
+        if ev:
+            ev[2].record(stream)
+        o = ulysses.head_to_seq(oh, w.Tq)
+        if ev:
+            ev[3].record(stream)
+        return o
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if h3.h3attn_check_status(ws, stream) != h3.OK:
+        raise RuntimeError("device status not OK after warm-up")
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        step(ev[i])
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    if h3.h3attn_check_status(ws, stream) != h3.OK:
+        raise RuntimeError("device status not OK after the timed steps")
+    total_ms = max_over_ranks(dist, ev[0][0].elapsed_time(ev[K - 1][3]), dev)
+    to_head = max_over_ranks(dist, statistics.mean(e[0].elapsed_time(e[1]) for e in ev), dev)
+    compute = max_over_ranks(dist, statistics.mean(e[1].elapsed_time(e[2]) for e in ev), dev)
+    to_seq = max_over_ranks(dist, statistics.mean(e[2].elapsed_time(e[3]) for e in ev), dev)
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    ms_step = total_ms / K
+    shard_bytes = 3 * w.B * counts[0] * w.H * w.D * 2  # Q, K and V of the largest token shard
+    cfg = config_of(w, world)
+    cfg["parallelism"] = (f"Ulysses over {world} GPU(s): token shards of {counts[-1]}-{counts[0]} tokens, "
+                          f"{hn} heads per GPU, NCCL all-to-all before and after")
+    line = {"metric": metric_of(w).replace("(1xB200)", f"({world}xB200, one sequence)"),
+            "value": w.ops / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic", "config": cfg,
+            "clocks": clk, "gpu_launches": launches_per_step(dataclasses.replace(w, H=hn)) * K,
+            "ulysses": {"seq_to_head_ms": to_head, "forward_ms": compute, "head_to_seq_ms": to_seq,
+                        "bytes_per_rank_to_head": shard_bytes, "bytes_per_rank_to_seq": shard_bytes // 3},
+            "e2e": None, "cpu_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------- latency mode ----
 def run_latency(args):
     """Per-call latency at the fixed shape (B1 H1 Tq128 Tkv192 D128), measured the way the
@@ -545,6 +654,8 @@ def main():
         w = dataclasses.replace(w, name=f"{w.name}_h{args.heads}", H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.ulysses:
+        run_ulysses(args, w)
     else:
         run_ours(args, w)
 

@@ -60,9 +60,11 @@ def seq_to_head(xs: Sequence[torch.Tensor], T: int, group=None) -> list:
             raise ValueError("the tensors of one exchange need one shape and dtype")
     Hn = H // world
     esz = xs[0].element_size()
-    # send buffer [N, n, B, T_r, Hn, D]: the block for rank d holds its heads of every tensor
-    stacked = torch.stack(list(xs))                                   # [n, B, T_r, H, D]
-    send = stacked.view(n, B, Tr, world, Hn, D).permute(3, 0, 1, 2, 4, 5).contiguous()
+    # send buffer [N, n, B, T_r, Hn, D]: the block for rank d holds its heads of every
+    # tensor (one strided copy per tensor)
+    send = torch.empty((world, n, B, Tr, Hn, D), dtype=xs[0].dtype, device=xs[0].device)
+    for i, x in enumerate(xs):
+        send[:, i].copy_(x.reshape(B, Tr, world, Hn, D).permute(2, 0, 1, 3, 4))
     recv = torch.empty(n * B * T * Hn * D * esz, dtype=torch.uint8, device=xs[0].device)
     dist.all_to_all_single(recv, _bytes(send), [n * B * c * Hn * D * esz for c in counts],
                            [n * B * Tr * Hn * D * esz] * world, group=group)
