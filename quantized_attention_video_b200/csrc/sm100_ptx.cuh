@@ -137,16 +137,6 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] x B[smem desc]^T, 8-bit signed integers, S32 accumulate.
-__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // D[tmem] (+)= A[smem desc] x B[smem desc]^T, E4M3 operands, F32 accumulate.
 __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -304,12 +294,9 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: D format in bits 4-5 (1 = F32, 2 = S32), A format in
-// 7-9, B format in 10-12 (8-bit integer: 1 = signed; FP8: 0 = E4M3; 16-bit: 1 = BF16), both
-// operands K-major (bits 15, 16 = 0), N >> 3 in 17-22, M >> 4 in 24-28.
-__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
+// Instruction descriptor: D format in bits 4-5 (1 = F32), A format in 7-9, B format in
+// 10-12 (FP8: 0 = E4M3; 16-bit: 1 = BF16), both operands K-major (bits 15, 16 = 0),
+// N >> 3 in 17-22, M >> 4 in 24-28.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
