@@ -164,11 +164,21 @@ h3attn_status h3attn_debug_qk_scores(const void* ws, size_t ws_bytes, int B, int
  * 0 for invalid sizes or heads_per_group outside [1, H]. */
 size_t h3attn_forward_host_bytes(int B, int Tq, int Tkv, int H, int D, int heads_per_group);
 
+/* The head groups of h3attn_forward_host(..., H, ..., heads_per_group): heads_per_group
+ * heads each, except that when H > 2 * heads_per_group (and heads_per_group >= 2) the
+ * first and the last group take heads_per_group / 2 heads.  Writes the first head of
+ * each group and then H to group_start[0 .. n] (n + 1 ints; NULL to only count, at most
+ * H + 1 entries are written) and returns the number of groups n; 0 for heads_per_group
+ * outside [1, H] or H outside [1, 4096]. */
+int h3attn_forward_host_groups(int H, int heads_per_group, int* group_start);
+
 /* Forward pass (as h3attn_forward_ex) from HOST input views to a HOST output view, for
  * callers whose activations are not resident on the device.  The heads are processed in
- * groups of heads_per_group: group g is uploaded on an internal stream, computed on
- * `stream`, and downloaded on a second internal stream, so the upload of group g+1 and
- * the download of group g-1 overlap the kernels of group g.  Heads are independent
+ * the groups of h3attn_forward_host_groups: group g is uploaded on an internal stream,
+ * computed on `stream`, and downloaded on a second internal stream, so the upload of
+ * group g+1 and the download of group g-1 overlap the kernels of group g.  Only the
+ * first group's upload and the last group's download stand alone, which is why those two
+ * groups are the smaller ones.  Heads are independent
  * problems (every statistic, scale and softmax is per (b, h)), so the result is bit for
  * bit that of one h3attn_forward_ex call on all heads.
  *   q, k, v, out: host views with the device views' rules (16-byte aligned data, strides
@@ -195,7 +205,8 @@ h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int
                                                int heads_per_group, void* stream);
 
 /* Failure-path test hook of the host pipeline: h3attn_forward_host with the attention of
- * head group fail_group (0 <= fail_group < ceil(H / heads_per_group)) launched through
+ * head group fail_group (0 <= fail_group < h3attn_forward_host_groups(H, heads_per_group,
+ * NULL)) launched through
  * h3attn_debug_attend_timeout (waits bounded by wait_limit_ns, 1 ms to 2 s, the O-ready
  * arrivals withheld), every other group as usual.  h3attn_forward_host_check_status then
  * reports H3ATTN_ERR_TIMEOUT, whichever group failed; the other groups' output heads are

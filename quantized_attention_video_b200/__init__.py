@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.h3attn_debug_attend_timeout.argtypes = [P, S] + [I] * 5 + [F, VP, ctypes.c_uint64, P]
         L.h3attn_forward_host_bytes.restype = S
         L.h3attn_forward_host_bytes.argtypes = [I] * 6
+        L.h3attn_forward_host_groups.restype = I
+        L.h3attn_forward_host_groups.argtypes = [I, I, P]
         L.h3attn_forward_host.restype = I
         L.h3attn_forward_host.argtypes = [VP, VP, VP] + [I] * 5 + [F, VP, I, P, S, P]
         L.h3attn_forward_host_check_status.restype = I
@@ -246,6 +248,16 @@ def h3attn_norm_rope(x, gamma, cos_tab, sin_tab, eps: float, out, stream=None):
 
 def h3attn_forward_host_bytes(B: int, Tq: int, Tkv: int, H: int, heads_per_group: int, D: int = HEAD_DIM) -> int:
     return lib().h3attn_forward_host_bytes(B, Tq, Tkv, H, D, heads_per_group)
+
+
+def h3attn_forward_host_groups(H: int, heads_per_group: int) -> list:
+    """First head of every head group of h3attn_forward_host, then H."""
+    n = lib().h3attn_forward_host_groups(H, heads_per_group, None)
+    if n == 0:
+        raise H3AttnError(ERR_INVALID_ARG, "h3attn_forward_host_groups")
+    buf = (ctypes.c_int * (n + 1))()
+    lib().h3attn_forward_host_groups(H, heads_per_group, buf)
+    return list(buf)
 
 
 def new_host_buffer(B: int, Tq: int, Tkv: int, H: int, heads_per_group: int, device="cuda"):

@@ -65,9 +65,41 @@ cudaError_t copy_heads(char* dev, const char* host, int64_t sb, int64_t st, int6
   return cudaSuccess;
 }
 
+// The head groups of a call: heads_per_group each, except that with more than
+// 2 * heads_per_group heads the first and the last group take heads_per_group / 2 (at
+// least 1).  Only the first group's upload and the last group's download are not
+// overlapped by kernels, so halving those two groups shortens the call.
+int group_starts(int H, int g, int* starts) {  // starts[0 .. n] with starts[n] = H; returns n
+  int n = 0, h = 0;
+  const int half = g / 2 > 0 ? g / 2 : 1;
+  const bool halved_ends = g >= 2 && H > 2 * g;
+  if (halved_ends) {
+    starts[n++] = 0;
+    h = half;
+  }
+  const int end = halved_ends ? H - half : H;
+  while (h < end) {
+    starts[n++] = h;
+    h += std::min(g, end - h);
+  }
+  if (halved_ends) starts[n++] = end;
+  starts[n] = H;
+  return n;
+}
+
 }  // namespace
 
 extern "C" {
+
+int h3attn_forward_host_groups(int H, int heads_per_group, int* group_start) {
+  if (H < 1 || heads_per_group < 1 || heads_per_group > H) return 0;
+  int tmp[4097];
+  if (H > 4096) return 0;
+  const int n = group_starts(H, heads_per_group, tmp);
+  if (group_start != nullptr)
+    for (int i = 0; i <= n; ++i) group_start[i] = tmp[i];
+  return n;
+}
 
 size_t h3attn_forward_host_bytes(int B, int Tq, int Tkv, int H, int D, int heads_per_group) {
   if (h3attn_workspace_bytes(B, Tq, Tkv, H, D) == 0) return 0;
@@ -103,7 +135,10 @@ h3attn_status forward_host_impl(const h3attn_bf16_view* q, const h3attn_bf16_vie
   if (dev_buf == nullptr || reinterpret_cast<uintptr_t>(dev_buf) % 1024 != 0 || dev_bytes < need)
     return H3ATTN_ERR_WORKSPACE;
 
-  const int g = heads_per_group, ngroups = (H + g - 1) / g;
+  const int g = heads_per_group;
+  if (H > 4096) return H3ATTN_ERR_INVALID_ARG;
+  int starts[4097];
+  const int ngroups = group_starts(H, g, starts);
   Slot sl{};
   if (!make_slot(B, Tq, Tkv, g, &sl)) return H3ATTN_ERR_INVALID_ARG;
   char* base = static_cast<char*>(dev_buf);
@@ -139,7 +174,7 @@ h3attn_status forward_host_impl(const h3attn_bf16_view* q, const h3attn_bf16_vie
   bool ok = cudaEventRecord(ev_start, cs) == cudaSuccess && cudaStreamWaitEvent(up, ev_start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(dn, ev_start, 0) == cudaSuccess;
   for (int gi = 0; ok && gi < ngroups; ++gi) {
-    const int slot = gi & 1, h0 = gi * g, gn = std::min(g, H - h0);
+    const int slot = gi & 1, h0 = starts[gi], gn = starts[gi + 1] - starts[gi];
     char* sb = base + (size_t)slot * sl.bytes;
     // upload: the slot's inputs are free once the forward pass of group gi-2 is done
     if (gi >= 2) ok = ok && cudaStreamWaitEvent(up, ev_comp[slot], 0) == cudaSuccess;
@@ -201,7 +236,7 @@ h3attn_status h3attn_debug_forward_host_timeout(const h3attn_bf16_view* q, const
                                                 float softmax_scale, const h3attn_bf16_out* out,
                                                 int heads_per_group, void* dev_buf, size_t dev_bytes,
                                                 int fail_group, uint64_t wait_limit_ns, void* stream) {
-  if (heads_per_group < 1 || fail_group < 0 || fail_group >= (H + heads_per_group - 1) / heads_per_group)
+  if (fail_group < 0 || fail_group >= h3attn_forward_host_groups(H, heads_per_group, nullptr))
     return H3ATTN_ERR_INVALID_ARG;
   return forward_host_impl(q, k, v, B, Tq, Tkv, H, D, softmax_scale, out, heads_per_group, dev_buf, dev_bytes,
                            stream, fail_group, wait_limit_ns);
@@ -214,7 +249,7 @@ h3attn_status h3attn_forward_host_check_status(void* dev_buf, int B, int Tq, int
   Slot sl{};
   if (!make_slot(B, Tq, Tkv, heads_per_group, &sl)) return H3ATTN_ERR_INVALID_ARG;
   h3attn_status first = H3ATTN_OK;
-  const int used = (H + heads_per_group - 1) / heads_per_group >= 2 ? 2 : 1;  // an unused slot holds no status
+  const int used = h3attn_forward_host_groups(H, heads_per_group, nullptr) >= 2 ? 2 : 1;  // an unused slot holds no status
   for (int slot = 0; slot < used; ++slot) {
     const h3attn_status st = h3attn_check_status(static_cast<char*>(dev_buf) + slot * sl.bytes + sl.ws, stream);
     if (first == H3ATTN_OK) first = st;

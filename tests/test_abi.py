@@ -161,3 +161,21 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "liboracle" not in text, fn
+
+
+def test_host_pipeline_group_layout(L):
+    """Groups of heads_per_group heads, the first and the last halved once there are more
+    than two full groups' worth of heads."""
+    assert h3.h3attn_forward_host_groups(32, 2) == [0] + list(range(1, 32, 2)) + [31, 32][1:]
+    assert h3.h3attn_forward_host_groups(8, 2) == [0, 1, 3, 5, 7, 8]
+    assert h3.h3attn_forward_host_groups(10, 3) == [0, 1, 4, 7, 9, 10]
+    assert h3.h3attn_forward_host_groups(4, 2) == [0, 2, 4]      # no room for halved ends
+    assert h3.h3attn_forward_host_groups(5, 1) == [0, 1, 2, 3, 4, 5]
+    assert h3.h3attn_forward_host_groups(7, 7) == [0, 7]
+    for H in range(1, 40):
+        for g in range(1, H + 1):
+            s = h3.h3attn_forward_host_groups(H, g)
+            sizes = [b - a for a, b in zip(s, s[1:])]
+            assert s[0] == 0 and s[-1] == H and all(1 <= n <= g for n in sizes), (H, g, s)
+    assert L.h3attn_forward_host_groups(8, 0, None) == 0
+    assert L.h3attn_forward_host_groups(8, 9, None) == 0

@@ -111,15 +111,17 @@ def test_status_is_sticky_across_later_calls():
 
 @pytest.mark.parametrize("fail_group", [0, 1, 2])
 def test_host_pipeline_reports_an_early_group_timeout(fail_group):
-    """h3attn_forward_host over 4 head groups (two device slots reused in turn) with the
-    waits of one early group withheld: h3attn_forward_host_check_status reports the
-    timeout although two later groups reused that group's slot; the heads of the other
-    groups are those of the normal pipeline."""
+    """h3attn_forward_host over 5 head groups of 1, 2, 2, 2 and 1 heads (two device slots
+    reused in turn) with the waits of one early group withheld:
+    h3attn_forward_host_check_status reports the timeout although later groups reused that
+    group's slot; the heads of the other groups are those of the normal pipeline."""
     w = synth.WORKLOADS["selfattn_h8_t4096"]
     x = synth.make_inputs(w)
     host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
     q, k, v = host(x["q"]), host(x["k"]), host(x["v"])
-    g = 2  # 8 heads -> 4 groups
+    g = 2
+    starts = h3.h3attn_forward_host_groups(w.H, g)
+    assert starts == [0, 1, 3, 5, 7, 8]  # halved first and last groups
     buf = h3.new_host_buffer(w.B, w.Tq, w.Tkv, w.H, g)
     ref = torch.empty(w.B, w.Tq, w.H, w.D, dtype=torch.bfloat16).pin_memory()
     h3.h3attn_forward_host(q, k, v, w.scale, ref, buf, g)
@@ -128,7 +130,7 @@ def test_host_pipeline_reports_an_early_group_timeout(fail_group):
     h3.h3attn_debug_forward_host_timeout(q, k, v, w.scale, out, buf, g, fail_group, LIMIT_NS)
     assert h3.h3attn_forward_host_check_status(buf, w.B, w.Tq, w.Tkv, w.H, g) == h3.ERR_TIMEOUT
     assert h3.h3attn_forward_host_check_status(buf, w.B, w.Tq, w.Tkv, w.H, g) == h3.OK
-    others = [h for h in range(w.H) if h // g != fail_group]
+    others = [h for h in range(w.H) if not starts[fail_group] <= h < starts[fail_group + 1]]
     assert torch.equal(out[:, :, others].view(torch.int16), ref[:, :, others].view(torch.int16))
 
 
