@@ -1,7 +1,7 @@
-"""The Ulysses exchange (quantized_attention_video_b200/ulysses.py) on two gloo ranks (CPU).
+"""The Ulysses exchange (quantized_attention_video_b200/ulysses.py) on gloo ranks (CPU).
 
-One sequence is spread over the ranks by tokens (ragged: 301 tokens give shards of 151
-and 150).  seq_to_head must hand every rank all tokens of its H/2 heads, head_to_seq
+One sequence is spread over two (or three) ranks by tokens (ragged: 301 tokens give
+shards of 151 and 150; 100 tokens over three ranks 34, 33 and 33).  seq_to_head must hand every rank all tokens of its H/2 heads, head_to_seq
 must invert it, and the composition with a per-head attention must give, on each
 rank's tokens, the bytes that one process computing every head produces.  The
 attention used here is the oracle's (the GPU library has no CPU path), so the
@@ -104,6 +104,36 @@ def test_two_ranks_give_the_single_process_bytes(tmp_path):
         assert np.array_equal(got, ref), name
     for r in range(world):
         assert open(tmp_path / f"errors{r}.txt").read().split("\n") == ["heads: refused", "tokens: refused"]
+
+
+def _rank_three(rank: int, world: int, port: int, out_dir: str):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        from quantized_attention_video_b200 import ulysses
+        w = synth.Workload("ulysses_b1_t100_h6", 1, 100, 100, 6, 128, "k_offset", 5103)
+        x = synth.make_inputs(w)
+        counts = ulysses.token_counts(w.Tq, world)
+        off = sum(counts[:rank])
+        q, k, v = (torch.from_numpy(np.ascontiguousarray(x[n][:, off:off + counts[rank]]).view(np.int16))
+                   for n in "qkv")
+        out = ulysses.ulysses_attention(q, k, v, w.Tq, w.scale, attend=_oracle_attention)
+        np.save(os.path.join(out_dir, f"three_out{rank}.npy"), out.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_ranks_with_a_ragged_split(tmp_path):
+    """100 tokens over three ranks (34, 33, 33), 6 heads (2 per rank)."""
+    world = 3
+    mp.start_processes(_rank_three, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    w = synth.Workload("ulysses_b1_t100_h6", 1, 100, 100, 6, 128, "k_offset", 5103)
+    x = synth.make_inputs(w)
+    ref = oracle.attend_all(oracle.quantize(x["q"], x["k"], x["v"]), w.scale, 128)
+    got = np.concatenate([np.load(tmp_path / f"three_out{r}.npy").view(np.uint16) for r in range(world)], axis=1)
+    assert [np.load(tmp_path / f"three_out{r}.npy").shape[1] for r in range(world)] == [34, 33, 33]
+    assert np.array_equal(got, ref)
 
 
 def test_token_counts_split_raggedly():
