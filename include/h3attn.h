@@ -187,6 +187,7 @@ int h3attn_forward_host_groups(int H, int heads_per_group, int* group_start);
  *     end of the call (every copy of the call is ordered before that point).
  *   dev_buf: device memory of h3attn_forward_host_bytes(...) bytes, 1024-byte aligned,
  *     owned by the caller; holds the staging and the per-slot workspaces.
+ *   H: at most 4096 (H3ATTN_ERR_INVALID_ARG beyond).
  * Asynchronous on `stream`; creates its two copy streams and eight events per call and
  * releases them before returning (the runtime frees them once their work is done).
  * Device-side status: h3attn_forward_host_check_status.  The zero-copy layout of
